@@ -1,0 +1,18 @@
+"""B200-native (sm_100a) additive, differentiable 2D Gaussian-splatting renderer.
+
+The hot path of "Learning Video Dynamics with Predictive Differentiable
+Rendering" (PDR): N anisotropic Gaussians per frame, each with 5 + C
+parameters, accumulated additively into a C-channel H x W field, forward and
+backward.  The kernels and their C ABI live in libpdr.so (include/pdr.h);
+this package is the thin PyTorch binding around it.
+"""
+from .api import (  # noqa: F401
+    Workspace,
+    bin_tiles,
+    list_capacity_per_frame,
+    render,
+    render_bwd,
+    render_fwd,
+    step_host,
+    workspace_bytes,
+)

@@ -1,0 +1,234 @@
+// C ABI of libpdr.so (declared in include/pdr.h): host-side validation,
+// geometry, workspace layout and kernel launches on the caller's stream.
+// The library allocates no device memory: everything lives in the caller's
+// workspace and buffers.
+#include <limits.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "pdr.h"
+
+namespace pdr {
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr size_t kScatterSmemLimit = 200 * 1024;
+constexpr int kBinTargetBlocks = 296;  // two binning blocks per SM on a 148-SM B200
+
+size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+
+int tiles_per_axis(int k) { return (k - 1 + kTile - 1) / kTile + 1; }
+
+struct Layout {
+    size_t err, gr, hist, offs, ids, total;
+};
+
+pdr_status make_geom(int B, int N, int C, int H, int W, int k, Geom *g) {
+    if (B < 1 || N < 1 || C < 1 || H < 1 || W < 1 || k < 1 || (k & 1) == 0)
+        return PDR_ERR_INVALID_ARG;
+    if (C > PDR_MAX_C || k > PDR_MAX_K) return PDR_ERR_TOO_LARGE;
+    const long long TX = (W + kTile - 1) / kTile, TY = (H + kTile - 1) / kTile;
+    const long long T = TX * TY;
+    if (T > PDR_MAX_TILES_PER_FRAME) return PDR_ERR_TOO_LARGE;
+    const long long m = tiles_per_axis(k);
+    const long long cap = (long long)N * m * m;
+    if ((long long)B * cap > INT_MAX || (long long)B * T > INT_MAX ||
+        (long long)B * N * (5 + C) > (long long)INT_MAX * 64)
+        return PDR_ERR_TOO_LARGE;
+    g->B = B; g->N = N; g->C = C; g->H = H; g->W = W; g->k = k; g->r = (k - 1) / 2;
+    g->TX = (int)TX; g->TY = (int)TY; g->T = (int)T;
+    g->P = 5 + C;
+    g->m = (int)m;
+    g->cap = (int)cap;
+    const long long total = (long long)B * N;
+    long long ch = (total + kBinTargetBlocks - 1) / kBinTargetBlocks;
+    ch = ((ch + 255) / 256) * 256;
+    if (ch < 256) ch = 256;
+    const long long nround = ((long long)N + 255) / 256 * 256;
+    if (ch > nround) ch = nround;
+    g->chunk = (int)ch;
+    g->nchunks = (int)(((long long)N + ch - 1) / ch);
+    int nw = 8;
+    while (nw > 1 && sizeof(int) * (size_t)T * (nw + 2) > kScatterSmemLimit) nw >>= 1;
+    if (sizeof(int) * (size_t)T * (nw + 2) > kScatterSmemLimit) return PDR_ERR_TOO_LARGE;
+    g->scatter_warps = nw;
+    g->out_vec2 = 0;
+    return PDR_OK;
+}
+
+Layout make_layout(const Geom &g) {
+    Layout L;
+    size_t o = 0;
+    L.err = o; o += align_up(sizeof(int));
+    L.gr = o; o += align_up(sizeof(float4) * 2 * (size_t)g.B * g.N);
+    L.hist = o; o += align_up(sizeof(int) * (size_t)g.B * g.nchunks * g.T);
+    L.offs = o; o += align_up(sizeof(int) * (size_t)g.B * (g.T + 1));
+    L.ids = o; o += align_up(sizeof(int) * (size_t)g.B * g.cap);
+    L.total = o;
+    return L;
+}
+
+Workspace carve(void *base, const Layout &L) {
+    char *p = static_cast<char *>(base);
+    Workspace w;
+    w.err = reinterpret_cast<int *>(p + L.err);
+    w.gr = reinterpret_cast<float4 *>(p + L.gr);
+    w.hist = reinterpret_cast<int *>(p + L.hist);
+    w.offs = reinterpret_cast<int *>(p + L.offs);
+    w.ids = reinterpret_cast<int *>(p + L.ids);
+    return w;
+}
+
+pdr_status check_ws(const Geom &g, void *ws, size_t bytes, Layout *L) {
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0) return PDR_ERR_INVALID_ARG;
+    *L = make_layout(g);
+    if (bytes < L->total) return PDR_ERR_WORKSPACE_TOO_SMALL;
+    return PDR_OK;
+}
+
+pdr_status from_cuda(cudaError_t e) { return e == cudaSuccess ? PDR_OK : PDR_ERR_CUDA; }
+
+bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3) == 0; }
+
+}  // namespace
+}  // namespace pdr
+
+using namespace pdr;
+
+extern "C" {
+
+int pdr_abi_version(void) { return 1; }
+
+const char *pdr_status_string(pdr_status s) {
+    switch (s) {
+        case PDR_OK: return "PDR_OK";
+        case PDR_ERR_INVALID_ARG: return "PDR_ERR_INVALID_ARG: bad size, even k, null or misaligned pointer";
+        case PDR_ERR_WORKSPACE_TOO_SMALL: return "PDR_ERR_WORKSPACE_TOO_SMALL";
+        case PDR_ERR_CUDA: return "PDR_ERR_CUDA: a CUDA call or kernel launch failed";
+        case PDR_ERR_DEVICE_TIMEOUT: return "PDR_ERR_DEVICE_TIMEOUT";
+        case PDR_ERR_INTERNAL: return "PDR_ERR_INTERNAL: a device-side check failed";
+        case PDR_ERR_TOO_LARGE: return "PDR_ERR_TOO_LARGE: sizes beyond the library limits";
+    }
+    return "unknown pdr_status";
+}
+
+size_t pdr_workspace_bytes(int B, int N, int C, int H, int W, int k) {
+    Geom g;
+    if (make_geom(B, N, C, H, W, k, &g) != PDR_OK) return 0;
+    return make_layout(g).total;
+}
+
+long long pdr_list_capacity_per_frame(int N, int k) {
+    if (N < 1 || k < 1 || (k & 1) == 0) return 0;
+    const long long m = tiles_per_axis(k);
+    return (long long)N * m * m;
+}
+
+pdr_status pdr_render_fwd(const float *params, int B, int N, int C, int H, int W, int k,
+                          float *image, void *workspace, size_t workspace_bytes,
+                          void *stream) {
+    Geom g;
+    pdr_status st = make_geom(B, N, C, H, W, k, &g);
+    if (st != PDR_OK) return st;
+    if (!params || !image || !aligned4(params) || !aligned4(image)) return PDR_ERR_INVALID_ARG;
+    Layout L;
+    st = check_ws(g, workspace, workspace_bytes, &L);
+    if (st != PDR_OK) return st;
+    const Workspace ws = carve(workspace, L);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    g.out_vec2 = ((g.W & 1) == 0) && ((reinterpret_cast<uintptr_t>(image) & 7) == 0);
+    st = from_cuda(launch_bin(params, g, ws, s));
+    if (st != PDR_OK) return st;
+    return from_cuda(launch_fwd(params, g, ws, image, s));
+}
+
+pdr_status pdr_render_bwd(const float *params, const float *grad_image, int B, int N, int C,
+                          int H, int W, int k, float *grad_params, void *workspace,
+                          size_t workspace_bytes, int workspace_holds_fwd_bins,
+                          void *stream) {
+    Geom g;
+    pdr_status st = make_geom(B, N, C, H, W, k, &g);
+    if (st != PDR_OK) return st;
+    if (!params || !grad_image || !grad_params || !aligned4(params) || !aligned4(grad_image) ||
+        !aligned4(grad_params))
+        return PDR_ERR_INVALID_ARG;
+    Layout L;
+    st = check_ws(g, workspace, workspace_bytes, &L);
+    if (st != PDR_OK) return st;
+    const Workspace ws = carve(workspace, L);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (!workspace_holds_fwd_bins) {
+        st = from_cuda(launch_bin(params, g, ws, s));
+        if (st != PDR_OK) return st;
+    }
+    return from_cuda(launch_bwd(params, grad_image, g, ws, grad_params, s));
+}
+
+pdr_status pdr_bin(const float *params, int B, int N, int C, int H, int W, int k,
+                   int *tile_offsets, int *tile_ids, void *workspace, size_t workspace_bytes,
+                   void *stream) {
+    Geom g;
+    pdr_status st = make_geom(B, N, C, H, W, k, &g);
+    if (st != PDR_OK) return st;
+    if (!params || !tile_offsets || !tile_ids || !aligned4(params)) return PDR_ERR_INVALID_ARG;
+    Layout L;
+    st = check_ws(g, workspace, workspace_bytes, &L);
+    if (st != PDR_OK) return st;
+    const Workspace ws = carve(workspace, L);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    st = from_cuda(launch_bin(params, g, ws, s));
+    if (st != PDR_OK) return st;
+    st = from_cuda(cudaMemcpyAsync(tile_offsets, ws.offs, sizeof(int) * (size_t)g.B * (g.T + 1),
+                                   cudaMemcpyDeviceToDevice, s));
+    if (st != PDR_OK) return st;
+    return from_cuda(cudaMemcpyAsync(tile_ids, ws.ids, sizeof(int) * (size_t)g.B * g.cap,
+                                     cudaMemcpyDeviceToDevice, s));
+}
+
+pdr_status pdr_step_host(const float *h_params, const float *h_grad_image, float *h_image,
+                         float *h_grad_params, int B, int N, int C, int H, int W, int k,
+                         float *d_params, float *d_grad_image, float *d_image,
+                         float *d_grad_params, void *workspace, size_t workspace_bytes,
+                         void *stream) {
+    Geom g;
+    pdr_status st = make_geom(B, N, C, H, W, k, &g);
+    if (st != PDR_OK) return st;
+    if (!h_params || !h_grad_image || !h_image || !h_grad_params || !d_params ||
+        !d_grad_image || !d_image || !d_grad_params)
+        return PDR_ERR_INVALID_ARG;
+    Layout L;
+    st = check_ws(g, workspace, workspace_bytes, &L);
+    if (st != PDR_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t pbytes = sizeof(float) * (size_t)B * N * g.P;
+    const size_t ibytes = sizeof(float) * (size_t)B * C * H * W;
+    st = from_cuda(cudaMemcpyAsync(d_params, h_params, pbytes, cudaMemcpyHostToDevice, s));
+    if (st != PDR_OK) return st;
+    st = from_cuda(cudaMemcpyAsync(d_grad_image, h_grad_image, ibytes, cudaMemcpyHostToDevice, s));
+    if (st != PDR_OK) return st;
+    st = pdr_render_fwd(d_params, B, N, C, H, W, k, d_image, workspace, workspace_bytes, stream);
+    if (st != PDR_OK) return st;
+    st = pdr_render_bwd(d_params, d_grad_image, B, N, C, H, W, k, d_grad_params, workspace,
+                        workspace_bytes, 1, stream);
+    if (st != PDR_OK) return st;
+    st = from_cuda(cudaMemcpyAsync(h_image, d_image, ibytes, cudaMemcpyDeviceToHost, s));
+    if (st != PDR_OK) return st;
+    return from_cuda(cudaMemcpyAsync(h_grad_params, d_grad_params, pbytes,
+                                     cudaMemcpyDeviceToHost, s));
+}
+
+pdr_status pdr_check_device_error(void *workspace, void *stream) {
+    if (!workspace) return PDR_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return PDR_ERR_CUDA;
+    int word = 0;
+    if (cudaMemcpy(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return PDR_ERR_CUDA;
+    if (word != 0) {
+        if (cudaMemset(workspace, 0, sizeof(int)) != cudaSuccess) return PDR_ERR_CUDA;
+        return PDR_ERR_INTERNAL;
+    }
+    return PDR_OK;
+}
+
+}  // extern "C"

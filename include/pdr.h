@@ -1,0 +1,146 @@
+/*
+ * pdr.h -- C ABI of libpdr.so: the additive, differentiable 2D Gaussian
+ * splatting renderer of "Learning Video Dynamics with Predictive
+ * Differentiable Rendering" (PDR), forward and backward, for NVIDIA B200
+ * (sm_100a).
+ *
+ * What is rendered (paper abstract: each Gaussian has "5 + C learnable
+ * parameters (position, scale, rotation, and C channel amplitudes)"; reading
+ * notes, "Method": the render is an additive accumulation; "Key Insight" and
+ * "Limitation": the kernel size / support is a tuned knob):
+ *
+ *     I_c(p) = sum_i a_ic * exp(-1/2 (p - mu_i)^T Sigma_i^{-1} (p - mu_i)),
+ *     Sigma_i = R(theta_i) diag(e^{2 s_i1}, e^{2 s_i2}) R(theta_i)^T,
+ *
+ * each Gaussian truncated to the k x k pixel window centred on round(mu_i)
+ * (ties round up), window pixels outside the grid dropped.  Pixel (x, y) sits
+ * at p = (x, y); x is the column, y the row; R(t) = [[cos t, -sin t],
+ * [sin t, cos t]].  No opacity, no compositing, no depth order.
+ *
+ * Layouts (all fp32, row-major, device memory unless stated):
+ *   params       [B][N][5+C]  per Gaussian (mu_x, mu_y, s_1, s_2, theta, a_0..a_{C-1})
+ *   image        [B][C][H][W]
+ *   grad_image   [B][C][H][W]  dL/dI
+ *   grad_params  [B][N][5+C]   dL/dparams, same order as params
+ *
+ * Ownership: the caller allocates every buffer, including the workspace
+ * (size from pdr_workspace_bytes); the library allocates no device memory.
+ * Outputs are overwritten, never accumulated into.
+ *
+ * Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ * stream).  All work is enqueued on it and the calls return without waiting.
+ * A PDR_ERR_CUDA return reports a launch error; errors during execution show
+ * up at the caller's next synchronisation.
+ *
+ * Validation (host side, before anything is launched; on failure nothing is
+ * launched and outputs are untouched): B, N, C, H, W >= 1; k odd and >= 1;
+ * sizes within the limits below (else PDR_ERR_TOO_LARGE); non-null pointers;
+ * workspace_bytes >= pdr_workspace_bytes(...) and a 256-byte aligned
+ * workspace.
+ *
+ * Numerics: fp32 arithmetic with a hardware base-2 exponential; fixed
+ * summation order (every list is in ascending Gaussian id), so results are
+ * bitwise reproducible run to run.  A Gaussian with a non-finite mean, or
+ * whose window misses the grid, contributes nothing and receives zero
+ * gradients; other non-finite parameters propagate NaN/Inf into that
+ * Gaussian's window pixels and its own gradients.  mu is clamped to
+ * [-2^24, 2^24] before the window centre is taken.  No gradient flows through
+ * round(mu) (the window position is piecewise constant in mu).
+ */
+#ifndef PDR_H
+#define PDR_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PDR_OK = 0,
+    PDR_ERR_INVALID_ARG = 1,          /* bad size, even k, null pointer, misaligned workspace */
+    PDR_ERR_WORKSPACE_TOO_SMALL = 2,  /* workspace_bytes < pdr_workspace_bytes(...) */
+    PDR_ERR_CUDA = 3,                 /* a CUDA runtime call or launch failed */
+    PDR_ERR_DEVICE_TIMEOUT = 4,       /* reserved: a bounded device-side wait gave up */
+    PDR_ERR_INTERNAL = 5,             /* a device-side consistency check failed */
+    PDR_ERR_TOO_LARGE = 6             /* sizes beyond the limits below */
+} pdr_status;
+
+/* Library limits (checked on the host). */
+#define PDR_TILE 16                    /* tile edge in pixels */
+#define PDR_MAX_C 8                    /* channels */
+#define PDR_MAX_K 31                   /* window size */
+#define PDR_MAX_TILES_PER_FRAME 16384  /* ceil(H/16) * ceil(W/16) */
+
+/* ABI version of this header (bumped on any incompatible change). */
+int pdr_abi_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *pdr_status_string(pdr_status s);
+
+/* Bytes of device workspace that pdr_render_fwd / pdr_render_bwd / pdr_bin
+ * need for these sizes; 0 if the sizes are invalid or beyond the limits.
+ * Computed on the host from a worst-case bound (every Gaussian touching the
+ * most tiles a k x k window can touch), so no device-to-host synchronisation
+ * is ever needed to size the tile lists. */
+size_t pdr_workspace_bytes(int B, int N, int C, int H, int W, int k);
+
+/* Forward render (abstract: "differentiable 2D Gaussian renderer supporting
+ * arbitrary channels"; reading notes, "Method": additive accumulation).
+ * Bins the Gaussians into 16x16 tiles (lists kept in the workspace) and
+ * writes image[B][C][H][W].  The bins stay valid in the workspace for a
+ * following pdr_render_bwd on the same params and sizes. */
+pdr_status pdr_render_fwd(const float *params, int B, int N, int C, int H, int W,
+                          int k, float *image, void *workspace,
+                          size_t workspace_bytes, void *stream);
+
+/* Backward pass: dL/dparams from dL/dI (abstract: "differentiable").
+ * grad_params[B][N][5+C] = (dL/dmu_x, dL/dmu_y, dL/ds_1, dL/ds_2,
+ * dL/dtheta, dL/da_0 .. dL/da_{C-1}) for every Gaussian.
+ * workspace_holds_fwd_bins = 1 reuses the bins a preceding pdr_render_fwd
+ * (or pdr_bin) left in this workspace for the same params and sizes;
+ * 0 re-bins first. */
+pdr_status pdr_render_bwd(const float *params, const float *grad_image, int B,
+                          int N, int C, int H, int W, int k, float *grad_params,
+                          void *workspace, size_t workspace_bytes,
+                          int workspace_holds_fwd_bins, void *stream);
+
+/* Tile binning only (exported for tests and tools).  Each frame b owns the
+ * list region [b * cap, (b + 1) * cap) of tile_ids, with
+ * cap = pdr_list_capacity_per_frame(N, k).  tile_offsets[b * (T + 1) + t] is
+ * the absolute start of tile t of frame b (T = tiles per frame, row-major);
+ * tile_offsets[b * (T + 1) + T] is the end of frame b's entries.  Entries are
+ * frame-local Gaussian indices, ascending within each tile.
+ * tile_offsets: [B * (T + 1)] int32, tile_ids: [B * cap] int32, device. */
+pdr_status pdr_bin(const float *params, int B, int N, int C, int H, int W, int k,
+                   int *tile_offsets, int *tile_ids, void *workspace,
+                   size_t workspace_bytes, void *stream);
+
+/* List capacity per frame used by pdr_bin: N times the most 16x16 tiles a
+ * k x k window can touch. */
+long long pdr_list_capacity_per_frame(int N, int k);
+
+/* One whole step from HOST memory, for callers whose data lives on the host:
+ * copies h_params and h_grad_image to the caller's device buffers d_params and
+ * d_grad_image, renders forward into d_image, runs the backward into
+ * d_grad_params, and copies the image and the gradients back to h_image and
+ * h_grad_params -- all enqueued on `stream` (one cudaMemcpyAsync per buffer;
+ * pinned host memory makes the copies asynchronous).  The call returns after
+ * enqueueing; synchronise the stream before reading h_image / h_grad_params. */
+pdr_status pdr_step_host(const float *h_params, const float *h_grad_image,
+                         float *h_image, float *h_grad_params, int B, int N,
+                         int C, int H, int W, int k, float *d_params,
+                         float *d_grad_image, float *d_image,
+                         float *d_grad_params, void *workspace,
+                         size_t workspace_bytes, void *stream);
+
+/* Synchronises `stream` and reports the device-side error word in the
+ * workspace (PDR_ERR_INTERNAL if a kernel's own bounds check fired), then
+ * clears it. */
+pdr_status pdr_check_device_error(void *workspace, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PDR_H */

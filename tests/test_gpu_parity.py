@@ -1,0 +1,202 @@
+"""CUDA path vs the fp64 oracle, through the C ABI (via the ctypes binding).
+
+Bars (normwise, per the stated tolerances): forward images within 1e-5 of
+max|I_ref| per (frame, channel); gradients within 1e-4 of max|ref| per
+parameter field (mu_x, mu_y, s_1, s_2, theta, each a_c) per frame; tile
+binning bit-exact.  Inputs are the seeded workloads of inputs.py plus edge
+cases (ties at .5, off-grid and non-finite means, k = 1, windows spanning
+three tiles, ragged grids, odd widths, long lists, C up to 8).
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from differentiable_gaussian_splatting_pdr_b200 import build as pdr_build
+from differentiable_gaussian_splatting_pdr_b200 import api as R
+from differentiable_gaussian_splatting_pdr_b200.inputs import (WORKLOADS, WORKLOAD_ORDER,
+                                                                Workload, make_inputs)
+
+pytestmark = pytest.mark.gpu
+
+FWD_TOL = 1e-5
+BWD_TOL = 1e-4
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    pdr_build.build()
+
+
+def threads():
+    return max(1, oracle.max_threads())
+
+
+def fwd_err(gpu: np.ndarray, ref: np.ndarray) -> float:
+    B, C = ref.shape[:2]
+    worst = 0.0
+    for b in range(B):
+        for c in range(C):
+            scale = np.abs(ref[b, c]).max()
+            err = np.abs(gpu[b, c].astype(np.float64) - ref[b, c]).max()
+            worst = max(worst, err / scale if scale > 0 else err)
+    return worst
+
+
+def bwd_err(gpu: np.ndarray, ref: np.ndarray) -> float:
+    B, N, P = ref.shape
+    worst = 0.0
+    for b in range(B):
+        for j in range(P):
+            scale = np.abs(ref[b, :, j]).max()
+            err = np.abs(gpu[b, :, j].astype(np.float64) - ref[b, :, j]).max()
+            worst = max(worst, err / scale if scale > 0 else err)
+    return worst
+
+
+def run_gpu(params: np.ndarray, grad: np.ndarray, H, W, k):
+    p = torch.from_numpy(params).cuda()
+    g = torch.from_numpy(grad).cuda()
+    img, ws = R.render_fwd(p, H, W, k)
+    dp = R.render_bwd(p, g, H, W, k, ws)
+    R.check_device_error(ws)
+    return img.cpu().numpy(), dp.cpu().numpy()
+
+
+def check_bins(params: np.ndarray, H, W, k):
+    p = torch.from_numpy(params).cuda()
+    offs, ids, cap = R.bin_tiles(p, H, W, k)
+    offs, ids = offs.cpu().numpy(), ids.cpu().numpy()
+    roffs, rids = oracle.bin_tiles(params, H, W, k)
+    B = params.shape[0]
+    T = offs.shape[1] - 1
+    for b in range(B):
+        frame_start = roffs[b * T]
+        assert offs[b, 0] == b * cap
+        for t in range(T):
+            got = ids[offs[b, t]:offs[b, t + 1]]
+            want = rids[roffs[b * T + t]:roffs[b * T + t + 1]]
+            assert np.array_equal(got, want), (b, t)
+        assert offs[b, T] - offs[b, 0] == roffs[(b + 1) * T] - frame_start
+
+
+def check_all(params, grad, H, W, k, bins=True):
+    if bins:
+        check_bins(params, H, W, k)
+    img, dp = run_gpu(params, grad, H, W, k)
+    ref_img = oracle.render_fwd(params, H, W, k, threads())
+    ref_dp = oracle.render_bwd(params, grad, H, W, k, threads())
+    ef, eb = fwd_err(img, ref_img), bwd_err(dp, ref_dp)
+    assert ef <= FWD_TOL, ef
+    assert eb <= BWD_TOL, eb
+    return ef, eb
+
+
+@pytest.mark.parametrize("name", WORKLOAD_ORDER)
+def test_workload_parity_full_size(name):
+    """Every workload at its full size: exact bins, all outputs vs the oracle."""
+    w = WORKLOADS[name]
+    p, g = make_inputs(w)
+    check_all(p, g, w.H, w.W, w.k)
+
+
+@pytest.mark.parametrize("name", ["tiny", "mono64", "rgb128"])
+def test_bitwise_reproducible(name):
+    w = WORKLOADS[name]
+    p, g = make_inputs(w)
+    a = run_gpu(p, g, w.H, w.W, w.k)
+    b = run_gpu(p, g, w.H, w.W, w.k)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+def _edge_params(rng, B, N, C, H, W, k, smean=0.4, ssd=0.4):
+    p = np.empty((B, N, 5 + C), dtype=np.float32)
+    p[..., 0] = rng.uniform(-k, W + k, (B, N))
+    p[..., 1] = rng.uniform(-k, H + k, (B, N))
+    p[..., 2] = rng.normal(smean, ssd, (B, N))
+    p[..., 3] = rng.normal(smean, ssd, (B, N))
+    p[..., 4] = rng.uniform(-7, 7, (B, N))
+    p[..., 5:] = rng.normal(0, 1, (B, N, C))
+    return p
+
+
+@pytest.mark.parametrize("B,N,C,H,W,k", [
+    (2, 300, 2, 40, 56, 17),    # windows spanning 2x2 tiles, ragged tiles
+    (1, 200, 1, 23, 37, 21),    # 3 tiles per axis, ragged both ways, odd width
+    (3, 150, 5, 48, 48, 31),    # largest window
+    (2, 100, 8, 33, 47, 9),     # C = 8, odd width
+    (1, 64, 3, 16, 16, 1),      # single-pixel windows
+    (4, 1, 4, 20, 30, 5),       # N = 1
+    (1, 500, 6, 7, 9, 3),       # grid smaller than a tile
+])
+def test_edge_shapes(B, N, C, H, W, k):
+    rng = np.random.default_rng(B * 1000 + N + C)
+    p = _edge_params(rng, B, N, C, H, W, k)
+    g = rng.standard_normal((B, C, H, W)).astype(np.float32)
+    check_all(p, g, H, W, k)
+
+
+def test_ties_offgrid_and_nonfinite_means():
+    rng = np.random.default_rng(7)
+    B, N, C, H, W, k = 1, 40, 2, 32, 48, 7
+    p = _edge_params(rng, B, N, C, H, W, k)
+    p[0, :8, 0] = [0.5, 15.5, np.nextafter(np.float32(16.5), np.float32(0)), -0.5, W - 0.5,
+                   np.float32(0.49999997), -3.4999, W + 2.5]
+    p[0, :8, 1] = [16.5, 0.5, 31.5, 2.5, -3.5, H - 0.5, 10.0, 5.0]
+    p[0, 8:12, 0] = [np.nan, np.inf, 1e30, -1e30]
+    p[0, 12:14, 1] = [np.nan, -np.inf]
+    g = rng.standard_normal((B, C, H, W)).astype(np.float32)
+    check_all(p, g, H, W, k)
+    _, dp = run_gpu(p, g, H, W, k)
+    assert np.all(dp[0, 8:14] == 0.0)
+
+
+def test_long_lists_in_one_tile():
+    """Thousands of Gaussians in one tile: several staging batches per block."""
+    rng = np.random.default_rng(8)
+    B, N, C, H, W, k = 2, 3000, 3, 32, 32, 9
+    p = _edge_params(rng, B, N, C, H, W, k)
+    p[..., 0] = rng.uniform(3, 12, (B, N))
+    p[..., 1] = rng.uniform(3, 12, (B, N))
+    g = rng.standard_normal((B, C, H, W)).astype(np.float32)
+    check_all(p, g, H, W, k)
+
+
+def test_autograd_matches_direct_calls():
+    w = WORKLOADS["mono64"].scaled(B=3)
+    p, g = make_inputs(w)
+    pt = torch.from_numpy(p).cuda().requires_grad_(True)
+    img = R.render(pt, w.H, w.W, w.k)
+    gt = torch.from_numpy(g).cuda()
+    (img * gt).sum().backward()
+    img2, dp2 = run_gpu(p, g, w.H, w.W, w.k)
+    assert np.array_equal(img.detach().cpu().numpy(), img2)
+    assert np.array_equal(pt.grad.cpu().numpy(), dp2)
+
+
+def test_host_step_matches_device_path():
+    w = WORKLOADS["rgb128"].scaled(B=2)
+    p, g = make_inputs(w)
+    hp = torch.from_numpy(p).pin_memory()
+    hg = torch.from_numpy(g).pin_memory()
+    h_img, h_dp, _ = R.step_host(hp, hg, w.H, w.W, w.k)
+    torch.cuda.synchronize()
+    img, dp = run_gpu(p, g, w.H, w.W, w.k)
+    assert np.array_equal(h_img.numpy(), img)
+    assert np.array_equal(h_dp.numpy(), dp)
+
+
+def test_invalid_arguments_rejected_on_device_buffers():
+    p = torch.zeros((1, 4, 6), device="cuda")
+    with pytest.raises(ValueError):
+        R.render_fwd(p, 16, 16, 4)
+    with pytest.raises(R._lib.PdrError):
+        lib = R._lib.load()
+        img = torch.empty((1, 1, 16, 16), device="cuda")
+        ws = torch.empty(16, dtype=torch.uint8, device="cuda")
+        R._lib.check("pdr_render_fwd", lib.pdr_render_fwd(
+            p.data_ptr(), 1, 4, 1, 16, 16, 5, img.data_ptr(), ws.data_ptr(), 16, None))
