@@ -1,0 +1,515 @@
+#!/usr/bin/env python
+"""Benchmark of the additive 2D Gaussian-splatting renderer, fwd + bwd.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...     # the fp64 CPU oracle on host cores
+
+One step = one pass of the whole hot path over one batch: tile binning, the
+forward render and the backward pass (dL/dI is a fixed synthetic N(0, 1)
+field, as in training after the loss).  The step is replayed from a CUDA
+graph (three library calls: bins, forward, backward, with timing-event nodes
+between them); L2 is flushed (a 256 MiB write) between timed steps, outside
+the timed events.  Each rank renders its own frames (weak scaling, no
+collective on the data path); the time is the max over ranks.
+
+Metric: Gaussian-pixel evaluations per second -- in-grid (Gaussian, window
+pixel) pairs of one pass, counted once per fwd + bwd step -- and frames/s.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from differentiable_gaussian_splatting_pdr_b200.inputs import (  # noqa: E402
+    WORKLOADS, WORKLOAD_ORDER, make_inputs, rank_seed)
+
+METRIC = "Gaussian-pixel evals/s and frames/s (fwd+bwd, 1 B200), % of roofline"
+UNIT = "evals/s"
+DEFAULT_WORKLOAD = "mono64"   # 16 frames, C=1, 64x64, N=1024/frame, k=9
+SM_COUNT = 148
+FP32_LANES_PER_SM = 128
+L2_FLUSH_BYTES = 256 << 20
+
+
+def fp32_ops_per_eval(C: int):
+    """Algorithmic FP32 instructions per in-window (Gaussian, pixel) pair:
+    forward 7 + C (offsets, quadratic form, C accumulations), backward 15 + 2C
+    (recompute 7, G = sum_c g_c a_c, v, C amplitude sums, five moments)."""
+    return 7 + C, 15 + 2 * C
+
+
+def in_grid_evals(params: np.ndarray, H: int, W: int, k: int) -> int:
+    """Number of in-grid (Gaussian, window pixel) pairs: the work unit."""
+    r = (k - 1) // 2
+    mu = params[..., :2].astype(np.float64)
+    ok = np.isfinite(mu).all(axis=-1)
+    c = np.floor(np.where(np.isfinite(mu), mu, 0.0) + 0.5)
+    nx = np.clip(np.minimum(c[..., 0] + r, W - 1) - np.maximum(c[..., 0] - r, 0) + 1, 0, None)
+    ny = np.clip(np.minimum(c[..., 1] + r, H - 1) - np.maximum(c[..., 1] - r, 0) + 1, 0, None)
+    return int((nx * ny * ok).sum())
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return json.load(f)
+    except OSError:
+        return {}
+
+
+def source_hash(*names) -> str:
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "differentiable_gaussian_splatting_pdr_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+KERNEL_SOURCES = {"k_fwd": ("render_fwd.cu", "common.cuh"), "k_bwd": ("render_bwd.cu", "common.cuh")}
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, or None
+    if there is none or the kernel source changed since it was captured."""
+    path = os.path.join(ROOT, "profiles", "%s_%s.md" % (kernel, workload))
+    try:
+        txt = open(path).read()
+    except OSError:
+        return None
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)\s+source_sha:\s*([0-9a-f]+)", txt)
+    if not m or m.group(2) != source_hash(*KERNEL_SOURCES[kernel]):
+        return None
+    return float(m.group(1))
+
+
+# ----------------------------------------------------------------------------
+# clocks
+# ----------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=5)
+        sm, mx, pw, reasons = [], [], [], set()
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+                pw.append(float(parts[3]))
+            except ValueError:
+                continue
+            for name, val in zip(self.NAMES, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "power_w_max": max(pw) if pw else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------
+# the oracle (CPU baseline and reference arm)
+# ----------------------------------------------------------------------------
+def oracle_sample(w, seconds: float, max_frames=None):
+    """Time the fp64 oracle fwd + bwd on the host cores over a bounded sample
+    of workload w: whole batches (or the first max_frames frames) repeated
+    until `seconds` have passed.  Returns (evals/s, frames/s, cores, sample)."""
+    import oracle  # test infrastructure: only the CPU-baseline leg runs it
+    B = w.B if max_frames is None else min(w.B, max_frames)
+    p, g = make_inputs(w)
+    p, g = p[:B].copy(), g[:B].copy()
+    ev = in_grid_evals(p, w.H, w.W, w.k)
+    cores = oracle.max_threads()
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.render_fwd(p, w.H, w.W, w.k, cores)
+        oracle.render_bwd(p, g, w.H, w.W, w.k, cores)
+        reps += 1
+        dt = time.perf_counter() - t0
+        if dt >= seconds:
+            break
+    sample = "%d x fwd+bwd of %d/%d frames of %s (%s)" % (reps, B, w.B, w.name, w.desc)
+    return ev * reps / dt, B * reps / dt, cores, sample, dt / reps
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return 0
+    import oracle
+    frames = w.B if w.name != "stress512" else 1
+    p, g = make_inputs(w)
+    p, g = p[:frames].copy(), g[:frames].copy()
+    ev = in_grid_evals(p, w.H, w.W, w.k)
+    cores = oracle.max_threads()
+    for _ in range(args.warmup):
+        oracle.render_fwd(p, w.H, w.W, w.k, cores)
+        oracle.render_bwd(p, g, w.H, w.W, w.k, cores)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.render_fwd(p, w.H, w.W, w.k, cores)
+        oracle.render_bwd(p, g, w.H, w.W, w.k, cores)
+        times.append(time.perf_counter() - t0)
+    tot = sum(times)
+    value = ev * len(times) / tot
+    sample = "%d frames of %s per step (%s), fp64 oracle, OpenMP over frames" % (frames, w.name, w.desc)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "frames_per_s": frames * len(times) / tot,
+        "config": workload_config(w, evals_per_step=ev, frames=frames),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w, **extra):
+    cfg = {"workload": w.name, "desc": w.desc, "B": w.B, "C": w.C, "H": w.H, "W": w.W,
+           "N": w.N, "k": w.k, "s": [w.s_mean, w.s_std], "amplitudes": list(w.amp),
+           "seed": w.seed}
+    cfg.update(extra)
+    return cfg
+
+
+# ----------------------------------------------------------------------------
+# the GPU arm
+# ----------------------------------------------------------------------------
+class Step:
+    """bins -> forward -> backward on one batch, captured in a CUDA graph with
+    timing events between the three library calls."""
+
+    def __init__(self, R, torch, w, seed, device):
+        self.R, self.torch, self.w, self.device = R, torch, w, device
+        p, g = make_inputs(w, seed)
+        self.evals = in_grid_evals(p, w.H, w.W, w.k)
+        self.h_params = torch.from_numpy(p).pin_memory()
+        self.h_grad = torch.from_numpy(g).pin_memory()
+        self.params = self.h_params.to(device)
+        self.grad = self.h_grad.to(device)
+        self.image = torch.empty((w.B, w.C, w.H, w.W), dtype=torch.float32, device=device)
+        self.dparams = torch.empty_like(self.params)
+        self.ws = R.Workspace.for_sizes(w.B, w.N, w.C, w.H, w.W, w.k, device)
+        self.ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
+        self.graph = None
+
+    def eager(self, events=None):
+        R, w = self.R, self.w
+        if events:
+            events[0].record()
+        R.build_bins(self.params, w.H, w.W, w.k, self.ws)
+        if events:
+            events[1].record()
+        R.render_fwd(self.params, w.H, w.W, w.k, self.ws, self.image, reuse_bins=True)
+        if events:
+            events[2].record()
+        R.render_bwd(self.params, self.grad, w.H, w.W, w.k, self.ws, self.dparams, reuse_bins=True)
+        if events:
+            events[3].record()
+
+    def capture(self):
+        torch = self.torch
+        s = torch.cuda.Stream(self.device)
+        s.wait_stream(torch.cuda.current_stream(self.device))
+        with torch.cuda.stream(s):
+            for _ in range(2):
+                self.eager()
+        torch.cuda.current_stream(self.device).wait_stream(s)
+        torch.cuda.synchronize(self.device)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self.eager(self.ev)
+        torch.cuda.synchronize(self.device)
+
+    def replay(self):
+        self.graph.replay()
+
+    def stage_ms(self):
+        e = self.ev
+        return (e[0].elapsed_time(e[3]), e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]),
+                e[2].elapsed_time(e[3]))
+
+
+def time_graph_steps(step, torch, flush, K, stream):
+    """K graph replays, L2 flushed before each; per-step (total, bins, fwd, bwd) ms."""
+    out = []
+    for _ in range(K):
+        flush.fill_(1)
+        step.replay()
+        stream.synchronize()
+        out.append(step.stage_ms())
+    return np.array(out)
+
+
+def time_eager_steps(step, torch, flush, K, stream):
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    out = []
+    for _ in range(K):
+        flush.fill_(1)
+        step.eager(ev)
+        stream.synchronize()
+        out.append(ev[0].elapsed_time(ev[3]))
+    return np.array(out)
+
+
+def time_e2e_steps(step, torch, K, stream):
+    """The host-buffer C-ABI call (pdr_step_host): H2D inputs, fwd, bwd, D2H
+    image and gradients, all inside the timed events."""
+    R, w = step.R, step.w
+    bufs = None
+    _, _, bufs = R.step_host(step.h_params, step.h_grad, w.H, w.W, w.k, None, step.device)
+    stream.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    out = []
+    for _ in range(K):
+        e0.record()
+        R.step_host(step.h_params, step.h_grad, w.H, w.W, w.k, bufs, step.device)
+        e1.record()
+        stream.synchronize()
+        out.append(e0.elapsed_time(e1))
+    h2d = step.h_params.numel() * 4 + step.h_grad.numel() * 4
+    d2h = bufs["h_image"].numel() * 4 + bufs["h_grad_params"].numel() * 4
+    return np.array(out), h2d, d2h
+
+
+def roofline_entry(kernel, ms, evals, C, peak_tops, workload, w):
+    ops_f, ops_b = fp32_ops_per_eval(C)
+    ops = evals * (ops_f if kernel == "k_fwd" else ops_b)
+    achieved = ops / (ms * 1e-3) / 1e12
+    if kernel == "k_fwd":
+        alg_bytes = 4 * w.B * w.N * (5 + C) + 4 * w.B * C * w.H * w.W
+    else:
+        alg_bytes = 8 * w.B * w.N * (5 + C) + 4 * w.B * C * w.H * w.W
+    return {"bound": "alu", "kernel": kernel, "achieved": achieved, "peak": peak_tops,
+            "unit": "Tinst/s", "frac": achieved / peak_tops,
+            "traffic": profiled_traffic(kernel, workload),
+            "ops_per_launch": ops, "algorithmic_bytes": alg_bytes,
+            "ms_per_launch": ms}
+
+
+def run_gpu(args, w):
+    import torch
+    import torch.distributed as dist
+    from differentiable_gaussian_splatting_pdr_b200 import api as R
+    from differentiable_gaussian_splatting_pdr_b200 import build as pdr_build
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print("warning: WORLD_SIZE=%d but --gpus %d" % (world, args.gpus), file=sys.stderr)
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+    if rank == 0:
+        pdr_build.build()
+    if world > 1:
+        dist.barrier()
+    R._lib.load()
+    stream = torch.cuda.current_stream(device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    step = Step(R, torch, w, rank_seed(w, rank), device)
+    step.capture()
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step.replay()
+    R.check_device_error(step.ws, device)
+
+    gpu_id = "GPU-" + str(torch.cuda.get_device_properties(device).uuid).replace("GPU-", "")
+    clocks = ClockSampler(gpu_id)
+    clocks.start()
+    t_soak = time.perf_counter()
+    while time.perf_counter() - t_soak < args.soak:   # clocks settle under the same step
+        flush.fill_(1)
+        step.replay()
+    stream.synchronize()
+
+    # ---------------- timed region ----------------
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    per = time_graph_steps(step, torch, flush, args.steps, stream)
+    torch.cuda.synchronize(device)
+    if world > 1:
+        dist.barrier()
+    # ----------------------------------------------
+    clk = clocks.stop()
+    R.check_device_error(step.ws, device)
+
+    total_ms = float(per[:, 0].sum())
+    t = torch.tensor([total_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_ms = float(t.item())
+    evals_all = step.evals * world
+    value = evals_all * args.steps / (max_ms * 1e-3)
+    frames_per_s = w.B * world * args.steps / (max_ms * 1e-3)
+
+    eager = time_eager_steps(step, torch, flush, args.steps, stream)
+    e2e, h2d, d2h = time_e2e_steps(step, torch, args.steps, stream)
+    te = torch.tensor([float(eager.sum()), float(e2e.sum())], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    eager_value = evals_all * args.steps / (float(te[0]) * 1e-3)
+    e2e_value = evals_all * args.steps / (float(te[1]) * 1e-3)
+
+    pk = measured_peaks()
+    sm_max = float(pk.get("sm_max_mhz") or 1965.0)
+    peak_tops = SM_COUNT * FP32_LANES_PER_SM * sm_max * 1e6 / 1e12
+    ms_bins, ms_fwd, ms_bwd = (float(np.mean(per[:, j])) for j in (1, 2, 3))
+    dominant = "k_bwd" if ms_bwd >= ms_fwd else "k_fwd"
+    roof = roofline_entry(dominant, ms_bwd if dominant == "k_bwd" else ms_fwd, step.evals,
+                          w.C, peak_tops, w.name, w)
+    roof["peak_source"] = ("148 SMs x 128 FP32 lanes x %.0f MHz (sm_max_mhz, MEASURED_PEAKS.json)"
+                           % sm_max)
+    other = roofline_entry("k_fwd" if dominant == "k_bwd" else "k_bwd",
+                           ms_fwd if dominant == "k_bwd" else ms_bwd, step.evals, w.C,
+                           peak_tops, w.name, w)
+
+    sweep = {}
+    if args.sweep and rank == 0:
+        for name in WORKLOAD_ORDER:
+            if name == w.name:
+                continue
+            sw = WORKLOADS[name]
+            st = Step(R, torch, sw, sw.seed, device)
+            st.capture()
+            for _ in range(5):
+                flush.fill_(1)
+                st.replay()
+            pr = time_graph_steps(st, torch, flush, args.sweep_steps, stream)
+            R.check_device_error(st.ws, device)
+            tot = float(pr[:, 0].mean())
+            f_ms, b_ms = float(pr[:, 2].mean()), float(pr[:, 3].mean())
+            of, ob = fp32_ops_per_eval(sw.C)
+            sweep[name] = {
+                "evals_per_s": st.evals / (tot * 1e-3), "frames_per_s": sw.B / (tot * 1e-3),
+                "ms_per_step": tot, "ms_bins": float(pr[:, 1].mean()), "ms_fwd": f_ms,
+                "ms_bwd": b_ms, "evals_per_step": st.evals,
+                "fwd_frac": st.evals * of / (f_ms * 1e-3) / 1e12 / peak_tops,
+                "bwd_frac": st.evals * ob / (b_ms * 1e-3) / 1e12 / peak_tops,
+                "step_frac": st.evals * (of + ob) / (tot * 1e-3) / 1e12 / peak_tops,
+            }
+            del st
+
+    cpu = None
+    if rank == 0 and world == 1 and args.cpu_seconds > 0:
+        v, fps, cores, sample, _ = oracle_sample(w, args.cpu_seconds)
+        cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
+               "frames_per_s": fps}
+
+    if rank == 0:
+        launches_per_step = 5   # k_count, k_scan, k_scatter, k_fwd, k_bwd
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": max_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic", "frames_per_s": frames_per_s,
+            "config": workload_config(
+                w, evals_per_step_per_gpu=step.evals, frames_per_gpu=w.B,
+                l2="flushed before every timed step (256 MiB write, outside the timed events)",
+                step="bins + forward + backward, CUDA-graph replay, per-step CUDA events",
+                parallelism="dp%d (frames sharded per rank, no data-path collective)" % world),
+            "roofline": roof,
+            "roofline_other_kernel": other,
+            "stages_ms": {"bins": ms_bins, "k_fwd": ms_fwd, "k_bwd": ms_bwd,
+                          "step": float(per[:, 0].mean())},
+            "eager": {"value": eager_value, "unit": UNIT,
+                      "note": "same step without graph replay (per-call launches)"},
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h,
+                    "api": "pdr_step_host: pinned host -> device, fwd, bwd, device -> host"},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk,
+            "cpu_baseline": cpu,
+            "sweep": sweep,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        del step
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=WORKLOAD_ORDER)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--soak", type=float, default=2.0,
+                    help="seconds of untimed steps while the clock sampler starts")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="host-core time budget of the oracle baseline (0 = skip)")
+    ap.add_argument("--no-sweep", dest="sweep", action="store_false")
+    ap.add_argument("--sweep-steps", type=int, default=50)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -9,6 +9,8 @@ this package is the thin PyTorch binding around it.
 from .api import (  # noqa: F401
     Workspace,
     bin_tiles,
+    build_bins,
+    check_device_error,
     list_capacity_per_frame,
     render,
     render_bwd,

@@ -30,7 +30,8 @@ SIGNATURES = {
     "pdr_status_string": (ctypes.c_char_p, [_i]),
     "pdr_workspace_bytes": (_sz, [_i] * 6),
     "pdr_list_capacity_per_frame": (_ll, [_i, _i]),
-    "pdr_render_fwd": (_i, [_vp] + [_i] * 6 + [_vp, _vp, _sz, _vp]),
+    "pdr_build_bins": (_i, [_vp] + [_i] * 6 + [_vp, _sz, _vp]),
+    "pdr_render_fwd": (_i, [_vp] + [_i] * 6 + [_vp, _vp, _sz, _i, _vp]),
     "pdr_render_bwd": (_i, [_vp, _vp] + [_i] * 6 + [_vp, _vp, _sz, _i, _vp]),
     "pdr_bin": (_i, [_vp] + [_i] * 6 + [_vp, _vp, _vp, _sz, _vp]),
     "pdr_step_host": (_i, [_vp, _vp, _vp, _vp] + [_i] * 6 + [_vp] * 5 + [_sz, _vp]),

@@ -71,19 +71,39 @@ def _workspace(ws, B, N, C, H, W, k, device) -> Workspace:
     return ws
 
 
-def render_fwd(params: torch.Tensor, H: int, W: int, k: int, workspace: Workspace | None = None,
-               out: torch.Tensor | None = None):
-    """Forward render; returns (image [B, C, H, W], workspace holding the bins)."""
+def build_bins(params: torch.Tensor, H: int, W: int, k: int,
+               workspace: Workspace | None = None) -> Workspace:
+    """Bin the Gaussians into 16x16 tiles inside a (new or given) workspace."""
     B, N, C = _check_params(params)
     dev = params.device
     ws = _workspace(workspace, B, N, C, H, W, k, dev)
+    lib = _lib.load()
+    _lib.check("pdr_build_bins", lib.pdr_build_bins(
+        _ptr(params), B, N, C, H, W, k, _ptr(ws.buf), ws.buf.numel(), _stream(dev)))
+    ws.shape = (B, N, C, H, W, k)
+    return ws
+
+
+def render_fwd(params: torch.Tensor, H: int, W: int, k: int, workspace: Workspace | None = None,
+               out: torch.Tensor | None = None, reuse_bins: bool = False):
+    """Forward render; returns (image [B, C, H, W], workspace holding the bins).
+
+    reuse_bins=True renders from the bins already in `workspace` (built by
+    build_bins or an earlier call on the same params and sizes)."""
+    B, N, C = _check_params(params)
+    dev = params.device
+    holds = bool(reuse_bins and workspace is not None and workspace.shape == (B, N, C, H, W, k))
+    ws = _workspace(workspace, B, N, C, H, W, k, dev)
+    if ws is not workspace:
+        holds = False
     if out is None:
         out = torch.empty((B, C, H, W), dtype=torch.float32, device=dev)
     elif out.shape != (B, C, H, W) or out.dtype != torch.float32 or not out.is_contiguous():
         raise ValueError("out must be contiguous fp32 [B, C, H, W]")
     lib = _lib.load()
     _lib.check("pdr_render_fwd", lib.pdr_render_fwd(
-        _ptr(params), B, N, C, H, W, k, _ptr(out), _ptr(ws.buf), ws.buf.numel(), _stream(dev)))
+        _ptr(params), B, N, C, H, W, k, _ptr(out), _ptr(ws.buf), ws.buf.numel(),
+        1 if holds else 0, _stream(dev)))
     ws.shape = (B, N, C, H, W, k)
     return out, ws
 

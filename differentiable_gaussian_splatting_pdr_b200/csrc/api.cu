@@ -124,9 +124,21 @@ long long pdr_list_capacity_per_frame(int N, int k) {
     return (long long)N * m * m;
 }
 
+pdr_status pdr_build_bins(const float *params, int B, int N, int C, int H, int W, int k,
+                          void *workspace, size_t workspace_bytes, void *stream) {
+    Geom g;
+    pdr_status st = make_geom(B, N, C, H, W, k, &g);
+    if (st != PDR_OK) return st;
+    if (!params || !aligned4(params)) return PDR_ERR_INVALID_ARG;
+    Layout L;
+    st = check_ws(g, workspace, workspace_bytes, &L);
+    if (st != PDR_OK) return st;
+    return from_cuda(launch_bin(params, g, carve(workspace, L), static_cast<cudaStream_t>(stream)));
+}
+
 pdr_status pdr_render_fwd(const float *params, int B, int N, int C, int H, int W, int k,
                           float *image, void *workspace, size_t workspace_bytes,
-                          void *stream) {
+                          int workspace_holds_bins, void *stream) {
     Geom g;
     pdr_status st = make_geom(B, N, C, H, W, k, &g);
     if (st != PDR_OK) return st;
@@ -137,8 +149,10 @@ pdr_status pdr_render_fwd(const float *params, int B, int N, int C, int H, int W
     const Workspace ws = carve(workspace, L);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     g.out_vec2 = ((g.W & 1) == 0) && ((reinterpret_cast<uintptr_t>(image) & 7) == 0);
-    st = from_cuda(launch_bin(params, g, ws, s));
-    if (st != PDR_OK) return st;
+    if (!workspace_holds_bins) {
+        st = from_cuda(launch_bin(params, g, ws, s));
+        if (st != PDR_OK) return st;
+    }
     return from_cuda(launch_fwd(params, g, ws, image, s));
 }
 
@@ -206,7 +220,8 @@ pdr_status pdr_step_host(const float *h_params, const float *h_grad_image, float
     if (st != PDR_OK) return st;
     st = from_cuda(cudaMemcpyAsync(d_grad_image, h_grad_image, ibytes, cudaMemcpyHostToDevice, s));
     if (st != PDR_OK) return st;
-    st = pdr_render_fwd(d_params, B, N, C, H, W, k, d_image, workspace, workspace_bytes, stream);
+    st = pdr_render_fwd(d_params, B, N, C, H, W, k, d_image, workspace, workspace_bytes, 0,
+                        stream);
     if (st != PDR_OK) return st;
     st = pdr_render_bwd(d_params, d_grad_image, B, N, C, H, W, k, d_grad_params, workspace,
                         workspace_bytes, 1, stream);

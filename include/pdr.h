@@ -85,21 +85,34 @@ const char *pdr_status_string(pdr_status s);
  * is ever needed to size the tile lists. */
 size_t pdr_workspace_bytes(int B, int N, int C, int H, int W, int k);
 
+/* Tile binning into the workspace (no rendering): every Gaussian enters the
+ * list of each 16x16 tile its clipped window touches, lists in ascending
+ * Gaussian id, together with a per-Gaussian record (window centre, rotated and
+ * scaled axes).  The window is the k x k "kernel support" of the reading
+ * notes ("Key Insight", "Limitation"); the ascending order gives every sum a
+ * fixed order (the additive accumulation itself has none).  The bins stay
+ * valid for pdr_render_fwd / pdr_render_bwd on the same params and sizes. */
+pdr_status pdr_build_bins(const float *params, int B, int N, int C, int H, int W,
+                          int k, void *workspace, size_t workspace_bytes,
+                          void *stream);
+
 /* Forward render (abstract: "differentiable 2D Gaussian renderer supporting
  * arbitrary channels"; reading notes, "Method": additive accumulation).
- * Bins the Gaussians into 16x16 tiles (lists kept in the workspace) and
- * writes image[B][C][H][W].  The bins stay valid in the workspace for a
+ * Writes image[B][C][H][W].  workspace_holds_bins = 1 uses the bins that
+ * pdr_build_bins (or a previous call) left in this workspace for the same
+ * params and sizes; 0 bins first.  The bins stay valid in the workspace for a
  * following pdr_render_bwd on the same params and sizes. */
 pdr_status pdr_render_fwd(const float *params, int B, int N, int C, int H, int W,
                           int k, float *image, void *workspace,
-                          size_t workspace_bytes, void *stream);
+                          size_t workspace_bytes, int workspace_holds_bins,
+                          void *stream);
 
 /* Backward pass: dL/dparams from dL/dI (abstract: "differentiable").
  * grad_params[B][N][5+C] = (dL/dmu_x, dL/dmu_y, dL/ds_1, dL/ds_2,
  * dL/dtheta, dL/da_0 .. dL/da_{C-1}) for every Gaussian.
- * workspace_holds_fwd_bins = 1 reuses the bins a preceding pdr_render_fwd
- * (or pdr_bin) left in this workspace for the same params and sizes;
- * 0 re-bins first. */
+ * workspace_holds_fwd_bins = 1 reuses the bins a preceding pdr_render_fwd,
+ * pdr_build_bins or pdr_bin left in this workspace for the same params and
+ * sizes; 0 re-bins first. */
 pdr_status pdr_render_bwd(const float *params, const float *grad_image, int B,
                           int N, int C, int H, int W, int k, float *grad_params,
                           void *workspace, size_t workspace_bytes,

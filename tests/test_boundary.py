@@ -95,15 +95,17 @@ FAKE = 0x10000
 def test_fwd_validation_order(lib):
     ws = lib.pdr_workspace_bytes(1, 64, 1, 32, 32, 7)
     f = lib.pdr_render_fwd
-    assert f(FAKE, 0, 64, 1, 32, 32, 7, FAKE, FAKE, ws, None) == 1
-    assert f(FAKE, 1, 64, 1, 32, 32, 6, FAKE, FAKE, ws, None) == 1
-    assert f(FAKE, 1, 64, 9, 32, 32, 7, FAKE, FAKE, ws, None) == 6
-    assert f(None, 1, 64, 1, 32, 32, 7, FAKE, FAKE, ws, None) == 1
-    assert f(FAKE, 1, 64, 1, 32, 32, 7, None, FAKE, ws, None) == 1
-    assert f(FAKE + 2, 1, 64, 1, 32, 32, 7, FAKE, FAKE, ws, None) == 1   # misaligned params
-    assert f(FAKE, 1, 64, 1, 32, 32, 7, FAKE, None, ws, None) == 1
-    assert f(FAKE, 1, 64, 1, 32, 32, 7, FAKE, FAKE + 16, ws, None) == 1  # workspace not 256-aligned
-    assert f(FAKE, 1, 64, 1, 32, 32, 7, FAKE, FAKE, ws - 1, None) == 2
+    assert f(FAKE, 0, 64, 1, 32, 32, 7, FAKE, FAKE, ws, 0, None) == 1
+    assert f(FAKE, 1, 64, 1, 32, 32, 6, FAKE, FAKE, ws, 0, None) == 1
+    assert f(FAKE, 1, 64, 9, 32, 32, 7, FAKE, FAKE, ws, 0, None) == 6
+    assert f(None, 1, 64, 1, 32, 32, 7, FAKE, FAKE, ws, 0, None) == 1
+    assert f(FAKE, 1, 64, 1, 32, 32, 7, None, FAKE, ws, 0, None) == 1
+    assert f(FAKE + 2, 1, 64, 1, 32, 32, 7, FAKE, FAKE, ws, 0, None) == 1   # misaligned params
+    assert f(FAKE, 1, 64, 1, 32, 32, 7, FAKE, None, ws, 0, None) == 1
+    assert f(FAKE, 1, 64, 1, 32, 32, 7, FAKE, FAKE + 16, ws, 0, None) == 1  # workspace not 256-aligned
+    assert f(FAKE, 1, 64, 1, 32, 32, 7, FAKE, FAKE, ws - 1, 0, None) == 2
+    assert lib.pdr_build_bins(FAKE, 1, 64, 1, 32, 32, 7, FAKE, ws - 1, None) == 2
+    assert lib.pdr_build_bins(None, 1, 64, 1, 32, 32, 7, FAKE, ws, None) == 1
 
 
 @no_gpu
@@ -132,7 +134,7 @@ def test_binding_fails_loudly_without_library(tmp_path):
 def test_python_api_surface():
     import differentiable_gaussian_splatting_pdr_b200 as pkg
     from differentiable_gaussian_splatting_pdr_b200 import api
-    for name in ["render", "render_fwd", "render_bwd", "bin_tiles", "step_host",
+    for name in ["render", "render_fwd", "render_bwd", "bin_tiles", "step_host", "build_bins",
                  "workspace_bytes", "check_device_error", "Workspace"]:
         assert callable(getattr(api, name)), name
     assert pkg.render is api.render

@@ -199,4 +199,17 @@ def test_invalid_arguments_rejected_on_device_buffers():
         img = torch.empty((1, 1, 16, 16), device="cuda")
         ws = torch.empty(16, dtype=torch.uint8, device="cuda")
         R._lib.check("pdr_render_fwd", lib.pdr_render_fwd(
-            p.data_ptr(), 1, 4, 1, 16, 16, 5, img.data_ptr(), ws.data_ptr(), 16, None))
+            p.data_ptr(), 1, 4, 1, 16, 16, 5, img.data_ptr(), ws.data_ptr(), 16, 0, None))
+
+
+def test_separate_bins_then_render_matches_one_call():
+    w = WORKLOADS["rgb128"].scaled(B=3)
+    p, g = make_inputs(w)
+    pt, gt = torch.from_numpy(p).cuda(), torch.from_numpy(g).cuda()
+    ws = R.build_bins(pt, w.H, w.W, w.k)
+    img, _ = R.render_fwd(pt, w.H, w.W, w.k, ws, reuse_bins=True)
+    dp = R.render_bwd(pt, gt, w.H, w.W, w.k, ws, reuse_bins=True)
+    R.check_device_error(ws)
+    img2, dp2 = run_gpu(p, g, w.H, w.W, w.k)
+    assert np.array_equal(img.cpu().numpy(), img2)
+    assert np.array_equal(dp.cpu().numpy(), dp2)
