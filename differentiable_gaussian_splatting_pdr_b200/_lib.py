@@ -36,6 +36,7 @@ SIGNATURES = {
     "pdr_bin": (_i, [_vp] + [_i] * 6 + [_vp, _vp, _vp, _sz, _vp]),
     "pdr_step_host": (_i, [_vp, _vp, _vp, _vp] + [_i] * 6 + [_vp] * 5 + [_sz, _vp]),
     "pdr_check_device_error": (_i, [_vp, _vp]),
+    "pdr_render_fwd_noalloc": (_i, [_vp] + [_i] * 6 + [_vp, _vp]),
 }
 
 _lib = None

@@ -147,6 +147,34 @@ pdr_status pdr_step_host(const float *h_params, const float *h_grad_image,
                          float *d_grad_params, void *workspace,
                          size_t workspace_bytes, void *stream);
 
+/* Bytes of the library's built-in device scratch (see pdr_render_fwd_noalloc). */
+#define PDR_STATIC_SCRATCH_BYTES (16u << 20)
+
+/* Forward render without any caller-provided workspace, for callers that
+ * cannot allocate device memory -- e.g. a plugin whose host application owns
+ * all device memory through its own pool, or a real-time loop that must not
+ * allocate after start-up.  The paper has no counterpart (this is an interface
+ * convenience, not a step of the method).
+ *
+ * Same inputs, output and numerics as pdr_render_fwd (params and image are the
+ * caller's device buffers); the bins live in a scratch array compiled into the
+ * library, PDR_STATIC_SCRATCH_BYTES (16 MiB) on every GPU that loads the
+ * library, held until the process exits.  Nothing is allocated: no
+ * cudaMalloc, cudaFree or allocating library routine.
+ *   - Sizes whose pdr_workspace_bytes(...) exceeds PDR_STATIC_SCRATCH_BYTES
+ *     (e.g. 16 frames of 64x64 with 1024 Gaussians each fit; 320 frames of
+ *     32x64 with 2048 each do not) return PDR_ERR_TOO_LARGE; bad sizes or null
+ *     pointers return PDR_ERR_INVALID_ARG; nothing is launched then.
+ *   - The first call made with a given device current looks up the scratch's
+ *     device address (cudaGetSymbolAddress) and caches it; make that first
+ *     call before any stream capture.
+ *   - All calls on a device share the one scratch, which keeps the last
+ *     call's contents.  Each call rebuilds everything it reads, so nothing
+ *     needs clearing, but calls that overlap on the GPU (other streams, other
+ *     host threads) race on it: serialise them. */
+pdr_status pdr_render_fwd_noalloc(const float *params, int B, int N, int C, int H,
+                                  int W, int k, float *image, void *stream);
+
 /* Synchronises `stream` and reports the device-side error word in the
  * workspace (PDR_ERR_INTERNAL if a kernel's own bounds check fired), then
  * clears it. */
