@@ -6,11 +6,13 @@
 
 One step = one pass of the whole hot path over one batch: tile binning, the
 forward render and the backward pass (dL/dI is a fixed synthetic N(0, 1)
-field, as in training after the loss).  The step is replayed from a CUDA
-graph (three library calls: bins, forward, backward, with timing-event nodes
-between them); L2 is flushed (a 256 MiB write) between timed steps, outside
-the timed events.  Each rank renders its own frames (weak scaling, no
-collective on the data path); the time is the max over ranks.
+field, as in training after the loss) -- two library calls, pdr_render_fwd
+(which bins) and pdr_render_bwd (which reuses the bins), replayed from a CUDA
+graph with a timing event on each side.  L2 is flushed (a 256 MiB write)
+between timed steps, outside the timed events.  Per-kernel times come from
+separate graphs with events between the calls, timed after the timed region.
+Each rank renders its own frames (weak scaling, no collective on the data
+path); the time is the max over ranks.
 
 Metric: Gaussian-pixel evaluations per second -- in-grid (Gaussian, window
 pixel) pairs of one pass, counted once per fwd + bwd step -- and frames/s.
@@ -228,9 +230,26 @@ def workload_config(w, **extra):
 # ----------------------------------------------------------------------------
 # the GPU arm
 # ----------------------------------------------------------------------------
+def graph_kernel_nodes(graph) -> int:
+    """Kernel nodes in a captured CUDA graph (all of them library kernels)."""
+    try:
+        from cuda.bindings import runtime as rt
+        g = rt.cudaGraph_t(init_value=graph.raw_cuda_graph())
+        err, _, n = rt.cudaGraphGetNodes(g, numNodes=0)
+        err, nodes, n = rt.cudaGraphGetNodes(g, numNodes=n)
+        kinds = [rt.cudaGraphNodeGetType(nd)[1] for nd in nodes]
+        return sum(1 for k in kinds if k == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel)
+    except Exception:  # pragma: no cover - reporting only
+        return -1
+
+
 class Step:
-    """bins -> forward -> backward on one batch, captured in a CUDA graph with
-    timing events between the three library calls."""
+    """One training-style pass on one batch: forward (binning included; for
+    frames of at most 16 tiles the binning runs inside the forward launch),
+    then the backward reusing the forward's bins.  Captured as CUDA graphs:
+      main  -- [event] forward, backward [event]           (the timed step)
+      split -- [event] forward [event] backward [event]    (stage times)
+      fwd   -- [event] bins [event] forward from bins [event] (k_fwd alone)"""
 
     def __init__(self, R, torch, w, seed, device):
         self.R, self.torch, self.w, self.device = R, torch, w, device
@@ -243,22 +262,37 @@ class Step:
         self.image = torch.empty((w.B, w.C, w.H, w.W), dtype=torch.float32, device=device)
         self.dparams = torch.empty_like(self.params)
         self.ws = R.Workspace.for_sizes(w.B, w.N, w.C, w.H, w.W, w.k, device)
-        self.ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
-        self.graph = None
+        self.graphs, self.events = {}, {}
 
-    def eager(self, events=None):
-        R, w = self.R, self.w
-        if events:
-            events[0].record()
-        R.build_bins(self.params, w.H, w.W, w.k, self.ws)
-        if events:
-            events[1].record()
-        R.render_fwd(self.params, w.H, w.W, w.k, self.ws, self.image, reuse_bins=True)
-        if events:
-            events[2].record()
-        R.render_bwd(self.params, self.grad, w.H, w.W, w.k, self.ws, self.dparams, reuse_bins=True)
-        if events:
-            events[3].record()
+    def fwd(self, reuse_bins=False):
+        w = self.w
+        self.R.render_fwd(self.params, w.H, w.W, w.k, self.ws, self.image, reuse_bins=reuse_bins)
+
+    def bwd(self):
+        w = self.w
+        self.R.render_bwd(self.params, self.grad, w.H, w.W, w.k, self.ws, self.dparams,
+                          reuse_bins=True)
+
+    def bins(self):
+        w = self.w
+        self.R.build_bins(self.params, w.H, w.W, w.k, self.ws)
+
+    def eager(self):
+        self.fwd()
+        self.bwd()
+
+    def _capture(self, name, parts):
+        torch = self.torch
+        ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(parts) + 1)]
+        g = torch.cuda.CUDAGraph(keep_graph=True)  # kept so its kernel nodes can be counted
+        with torch.cuda.graph(g):
+            ev[0].record()
+            for j, part in enumerate(parts):
+                for fn in part:
+                    fn()
+                ev[j + 1].record()
+        g.instantiate()
+        self.graphs[name], self.events[name] = g, ev
 
     def capture(self):
         torch = self.torch
@@ -267,41 +301,45 @@ class Step:
         with torch.cuda.stream(s):
             for _ in range(2):
                 self.eager()
+                self.bins()
+                self.fwd(reuse_bins=True)
         torch.cuda.current_stream(self.device).wait_stream(s)
         torch.cuda.synchronize(self.device)
-        self.graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(self.graph):
-            self.eager(self.ev)
+        self._capture("main", [[self.fwd, self.bwd]])
+        self._capture("split", [[self.fwd], [self.bwd]])
+        self._capture("fwd", [[self.bins], [lambda: self.fwd(reuse_bins=True)]])
         torch.cuda.synchronize(self.device)
 
-    def replay(self):
-        self.graph.replay()
+    def replay(self, name="main"):
+        self.graphs[name].replay()
 
-    def stage_ms(self):
-        e = self.ev
-        return (e[0].elapsed_time(e[3]), e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]),
-                e[2].elapsed_time(e[3]))
+    def times(self, name):
+        e = self.events[name]
+        return [e[j].elapsed_time(e[j + 1]) for j in range(len(e) - 1)]
 
 
-def time_graph_steps(step, torch, flush, K, stream):
-    """K graph replays, L2 flushed before each; per-step (total, bins, fwd, bwd) ms."""
+def time_graph(step, name, flush, K, stream):
+    """K replays of one graph, L2 flushed before each; per-step [total, stages...] ms."""
     out = []
     for _ in range(K):
         flush.fill_(1)
-        step.replay()
+        step.replay(name)
         stream.synchronize()
-        out.append(step.stage_ms())
+        st = step.times(name)
+        out.append([sum(st)] + st)
     return np.array(out)
 
 
 def time_eager_steps(step, torch, flush, K, stream):
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     out = []
     for _ in range(K):
         flush.fill_(1)
-        step.eager(ev)
+        e0.record()
+        step.eager()
+        e1.record()
         stream.synchronize()
-        out.append(ev[0].elapsed_time(ev[3]))
+        out.append(e0.elapsed_time(e1))
     return np.array(out)
 
 
@@ -385,7 +423,7 @@ def run_gpu(args, w):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(device)
-    per = time_graph_steps(step, torch, flush, args.steps, stream)
+    per = time_graph(step, "main", flush, args.steps, stream)
     torch.cuda.synchronize(device)
     if world > 1:
         dist.barrier()
@@ -410,10 +448,17 @@ def run_gpu(args, w):
     eager_value = evals_all * args.steps / (float(te[0]) * 1e-3)
     e2e_value = evals_all * args.steps / (float(te[1]) * 1e-3)
 
+    # Stage breakdown (after the timed region, same L2 flushing).
+    split = time_graph(step, "split", flush, args.steps, stream)
+    fsplit = time_graph(step, "fwd", flush, args.steps, stream)
+    ms_fwd_step = float(np.mean(split[:, 1]))     # forward incl. binning, as in the step
+    ms_bwd = float(np.mean(split[:, 2]))          # k_bwd alone
+    ms_bins = float(np.mean(fsplit[:, 1]))        # binning alone
+    ms_fwd = float(np.mean(fsplit[:, 2]))         # k_fwd alone, from prebuilt bins
+
     pk = measured_peaks()
     sm_max = float(pk.get("sm_max_mhz") or 1965.0)
     peak_tops = SM_COUNT * FP32_LANES_PER_SM * sm_max * 1e6 / 1e12
-    ms_bins, ms_fwd, ms_bwd = (float(np.mean(per[:, j])) for j in (1, 2, 3))
     dominant = "k_bwd" if ms_bwd >= ms_fwd else "k_fwd"
     roof = roofline_entry(dominant, ms_bwd if dominant == "k_bwd" else ms_fwd, step.evals,
                           w.C, peak_tops, w.name, w)
@@ -434,15 +479,19 @@ def run_gpu(args, w):
             for _ in range(5):
                 flush.fill_(1)
                 st.replay()
-            pr = time_graph_steps(st, torch, flush, args.sweep_steps, stream)
+            pr = time_graph(st, "main", flush, args.sweep_steps, stream)
+            sp = time_graph(st, "split", flush, args.sweep_steps, stream)
+            fs = time_graph(st, "fwd", flush, args.sweep_steps, stream)
             R.check_device_error(st.ws, device)
             tot = float(pr[:, 0].mean())
-            f_ms, b_ms = float(pr[:, 2].mean()), float(pr[:, 3].mean())
+            f_ms, b_ms = float(fs[:, 2].mean()), float(sp[:, 2].mean())
             of, ob = fp32_ops_per_eval(sw.C)
             sweep[name] = {
                 "evals_per_s": st.evals / (tot * 1e-3), "frames_per_s": sw.B / (tot * 1e-3),
-                "ms_per_step": tot, "ms_bins": float(pr[:, 1].mean()), "ms_fwd": f_ms,
+                "ms_per_step": tot, "ms_fwd_incl_bins": float(sp[:, 1].mean()),
+                "ms_bins": float(fs[:, 1].mean()), "ms_fwd": f_ms,
                 "ms_bwd": b_ms, "evals_per_step": st.evals,
+                "kernels_per_step": graph_kernel_nodes(st.graphs["main"]),
                 "fwd_frac": st.evals * of / (f_ms * 1e-3) / 1e12 / peak_tops,
                 "bwd_frac": st.evals * ob / (b_ms * 1e-3) / 1e12 / peak_tops,
                 "step_frac": st.evals * (of + ob) / (tot * 1e-3) / 1e12 / peak_tops,
@@ -456,7 +505,7 @@ def run_gpu(args, w):
                "frames_per_s": fps}
 
     if rank == 0:
-        launches_per_step = 5   # k_count, k_scan, k_scatter, k_fwd, k_bwd
+        launches_per_step = graph_kernel_nodes(step.graphs["main"])
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": max_ms / args.steps,
@@ -465,12 +514,14 @@ def run_gpu(args, w):
             "config": workload_config(
                 w, evals_per_step_per_gpu=step.evals, frames_per_gpu=w.B,
                 l2="flushed before every timed step (256 MiB write, outside the timed events)",
-                step="bins + forward + backward, CUDA-graph replay, per-step CUDA events",
+                step="forward (with its binning) + backward, CUDA-graph replay, per-step CUDA events",
                 parallelism="dp%d (frames sharded per rank, no data-path collective)" % world),
             "roofline": roof,
             "roofline_other_kernel": other,
-            "stages_ms": {"bins": ms_bins, "k_fwd": ms_fwd, "k_bwd": ms_bwd,
-                          "step": float(per[:, 0].mean())},
+            "stages_ms": {"step": float(per[:, 0].mean()), "fwd_incl_bins": ms_fwd_step,
+                          "k_bwd": ms_bwd, "bins_alone": ms_bins, "k_fwd_alone": ms_fwd,
+                          "note": "step = forward (binning inside) + backward, one graph; "
+                                  "the other figures come from split graphs timed after it"},
             "eager": {"value": eager_value, "unit": UNIT,
                       "note": "same step without graph replay (per-call launches)"},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,

@@ -13,7 +13,7 @@ namespace {
 
 constexpr size_t kAlign = 256;
 constexpr size_t kScatterSmemLimit = 200 * 1024;
-constexpr int kBinTargetBlocks = 296;  // two binning blocks per SM on a 148-SM B200
+constexpr int kScatterWarps = 8;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 
@@ -32,7 +32,7 @@ pdr_status make_geom(int B, int N, int C, int H, int W, int k, Geom *g) {
     if (T > PDR_MAX_TILES_PER_FRAME) return PDR_ERR_TOO_LARGE;
     const long long m = tiles_per_axis(k);
     const long long cap = (long long)N * m * m;
-    if ((long long)B * cap > INT_MAX || (long long)B * T > INT_MAX ||
+    if ((long long)B * cap > INT_MAX || (long long)B * T > INT_MAX || B > 65535 ||
         (long long)B * N * (5 + C) > (long long)INT_MAX * 64)
         return PDR_ERR_TOO_LARGE;
     g->B = B; g->N = N; g->C = C; g->H = H; g->W = W; g->k = k; g->r = (k - 1) / 2;
@@ -40,19 +40,22 @@ pdr_status make_geom(int B, int N, int C, int H, int W, int k, Geom *g) {
     g->P = 5 + C;
     g->m = (int)m;
     g->cap = (int)cap;
-    const long long total = (long long)B * N;
-    long long ch = (total + kBinTargetBlocks - 1) / kBinTargetBlocks;
-    ch = ((ch + 255) / 256) * 256;
-    if (ch < 256) ch = 256;
-    const long long nround = ((long long)N + 255) / 256 * 256;
-    if (ch > nround) ch = nround;
-    g->chunk = (int)ch;
-    g->nchunks = (int)(((long long)N + ch - 1) / ch);
-    int nw = 8;
+    g->nchunks = (N + kBinChunk - 1) / kBinChunk;
+    int nw = kScatterWarps;  // scatter block: as many warps as the per-warp tile masks allow
     while (nw > 1 && sizeof(int) * (size_t)T * (nw + 2) > kScatterSmemLimit) nw >>= 1;
     if (sizeof(int) * (size_t)T * (nw + 2) > kScatterSmemLimit) return PDR_ERR_TOO_LARGE;
     g->scatter_warps = nw;
+    // Small frames: one binning block per frame (its shared-memory tables
+    // hold [2 + 2 * warps] x T ints).
+    g->frame_block = T <= kFrameBlockMaxT && N <= kFrameBlockMaxN;
+    int ft = ((N + 31) / 32) * 32;
+    if (ft > 1024) ft = 1024;
+    if (B > 148 && ft > 512) ft = 512;  // more frames than SMs: more, smaller blocks
+    g->frame_threads = ft;
+    g->cluster_fwd = T <= kClusterTiles;
+    g->fwd_pl = (long long)B * T <= 2368 ? 2 : 4;  // small grids: more, shorter lanes per tile
     g->out_vec2 = 0;
+    g->out_vec4 = 0;
     return PDR_OK;
 }
 
@@ -87,6 +90,10 @@ pdr_status check_ws(const Geom &g, void *ws, size_t bytes, Layout *L) {
 }
 
 pdr_status from_cuda(cudaError_t e) { return e == cudaSuccess ? PDR_OK : PDR_ERR_CUDA; }
+
+cudaError_t bin(const float *params, const Geom &g, const Workspace &ws, cudaStream_t s) {
+    return launch_bin(params, g, ws, s);
+}
 
 bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3) == 0; }
 
@@ -133,7 +140,7 @@ pdr_status pdr_build_bins(const float *params, int B, int N, int C, int H, int W
     Layout L;
     st = check_ws(g, workspace, workspace_bytes, &L);
     if (st != PDR_OK) return st;
-    return from_cuda(launch_bin(params, g, carve(workspace, L), static_cast<cudaStream_t>(stream)));
+    return from_cuda(bin(params, g, carve(workspace, L), static_cast<cudaStream_t>(stream)));
 }
 
 pdr_status pdr_render_fwd(const float *params, int B, int N, int C, int H, int W, int k,
@@ -149,11 +156,14 @@ pdr_status pdr_render_fwd(const float *params, int B, int N, int C, int H, int W
     const Workspace ws = carve(workspace, L);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     g.out_vec2 = ((g.W & 1) == 0) && ((reinterpret_cast<uintptr_t>(image) & 7) == 0);
+    g.out_vec4 = ((g.W & 3) == 0) && ((reinterpret_cast<uintptr_t>(image) & 15) == 0);
+    if (!workspace_holds_bins && g.cluster_fwd)  // small frames: bins + render, one launch
+        return from_cuda(launch_fwd(params, g, ws, image, s, true));
     if (!workspace_holds_bins) {
-        st = from_cuda(launch_bin(params, g, ws, s));
+        st = from_cuda(bin(params, g, ws, s));
         if (st != PDR_OK) return st;
     }
-    return from_cuda(launch_fwd(params, g, ws, image, s));
+    return from_cuda(launch_fwd(params, g, ws, image, s, false));
 }
 
 pdr_status pdr_render_bwd(const float *params, const float *grad_image, int B, int N, int C,
@@ -172,7 +182,7 @@ pdr_status pdr_render_bwd(const float *params, const float *grad_image, int B, i
     const Workspace ws = carve(workspace, L);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (!workspace_holds_fwd_bins) {
-        st = from_cuda(launch_bin(params, g, ws, s));
+        st = from_cuda(bin(params, g, ws, s));
         if (st != PDR_OK) return st;
     }
     return from_cuda(launch_bwd(params, grad_image, g, ws, grad_params, s));
@@ -190,7 +200,7 @@ pdr_status pdr_bin(const float *params, int B, int N, int C, int H, int W, int k
     if (st != PDR_OK) return st;
     const Workspace ws = carve(workspace, L);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    st = from_cuda(launch_bin(params, g, ws, s));
+    st = from_cuda(bin(params, g, ws, s));
     if (st != PDR_OK) return st;
     st = from_cuda(cudaMemcpyAsync(tile_offsets, ws.offs, sizeof(int) * (size_t)g.B * (g.T + 1),
                                    cudaMemcpyDeviceToDevice, s));

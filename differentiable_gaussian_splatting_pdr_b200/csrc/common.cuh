@@ -14,6 +14,7 @@ constexpr int kNoCenter = 0x40000000;
 // Bits of the device error word (workspace), set by the kernels' own checks.
 constexpr int kErrListBounds = 1;  // a tile list or list slot outside its frame's region
 constexpr int kErrBadId = 2;       // a list entry that is not a Gaussian of the frame
+constexpr int kErrSmemLayout = 4;  // a kernel got less dynamic shared memory than it lays out
 
 // sqrt(kappa) with kappa = log2(e) / 2: scaling u by sqrt(kappa e^{-2 s})
 // turns exp(-q / 2) into 2^{-(u1^2 + u2^2)}.
@@ -27,10 +28,20 @@ struct Geom {
     int P;              // parameters per Gaussian (5 + C)
     int m;              // most tiles a window can touch along one axis
     int cap;            // tile-list capacity per frame (N * m * m)
-    int chunk, nchunks; // Gaussians per binning chunk, chunks per frame
+    int nchunks;        // binning chunks per frame (kBinChunk Gaussians each)
     int scatter_warps;  // warps per scatter block
-    int out_vec2;       // 1 if the output image allows 8-byte pixel-pair stores
+    int frame_block;    // 1: small frames, one binning block per frame
+    int frame_threads;  // threads of that block
+    int cluster_fwd;    // 1: frames of <= kClusterTiles tiles, bins + forward in one launch
+    int fwd_pl;         // forward pixels per lane (2 or 4)
+    int out_vec2;       // 1 if the output image allows 8-byte 2-pixel stores
+    int out_vec4;       // 1 if the output image allows 16-byte 4-pixel stores
 };
+
+constexpr int kBinChunk = 1024;        // Gaussians per binning block (large frames)
+constexpr int kFrameBlockMaxT = 256;   // small frames: at most this many tiles
+constexpr int kFrameBlockMaxN = 16384; // and at most this many Gaussians
+constexpr int kClusterTiles = 16;      // frames up to this many tiles: one cluster per frame
 
 // Per-Gaussian record written by the binner and read by both render kernels
 // (two float4 per Gaussian, 32 bytes):
@@ -42,7 +53,7 @@ struct Geom {
 struct Workspace {
     int *err;       // device error word
     float4 *gr;     // [B*N][2]
-    int *hist;      // [B][nchunks][T]: chunk counts, then absolute list bases
+    int *hist;      // [B][nchunks][T]: chunk counts, then prefix over chunks
     int *offs;      // [B][T + 1]: absolute list start of every tile, frame end
     int *ids;       // [B][cap]: frame-local Gaussian ids, tile-major
 };
@@ -69,11 +80,64 @@ __device__ __forceinline__ int round_half_up(float mu) {
     return (int)c;
 }
 
+// The per-Gaussian record (layout above) from its parameters.  One function
+// for the binner and for the render kernels that find their Gaussians
+// themselves, so both paths produce the same bits.
+__device__ __forceinline__ void gaussian_record(const float *__restrict__ p, float4 &A,
+                                                float4 &Q) {
+    const float mx = p[0], my = p[1], s1 = p[2], s2 = p[3], th = p[4];
+    int cx = kNoCenter, cy = kNoCenter;
+    if (isfinite(mx) && isfinite(my)) {
+        cx = round_half_up(mx);
+        cy = round_half_up(my);
+    }
+    float sn, cs;
+    sincosf(th, &sn, &cs);
+    const float h1 = kSqrtKappa * expf(-s1), h2 = kSqrtKappa * expf(-s2);
+    A = make_float4(mx, my, h1 * cs, h1 * sn);
+    Q = make_float4(-h2 * sn, h2 * cs, __int_as_float(cx), __int_as_float(cy));
+}
+
+// Window centre of a Gaussian from its mean alone (as in gaussian_record).
+__device__ __forceinline__ void window_centre(const float *__restrict__ p, int &cx, int &cy) {
+    const float mx = p[0], my = p[1];
+    cx = kNoCenter;
+    cy = kNoCenter;
+    if (isfinite(mx) && isfinite(my)) {
+        cx = round_half_up(mx);
+        cy = round_half_up(my);
+    }
+}
+
+// The window clipped to the grid; false if it misses the grid.
+__device__ __forceinline__ bool window_rect(int cx, int cy, const Geom &g, int &x0, int &x1,
+                                            int &y0, int &y1) {
+    x0 = max(cx - g.r, 0);
+    x1 = min(cx + g.r, g.W - 1);
+    y0 = max(cy - g.r, 0);
+    y1 = min(cy + g.r, g.H - 1);
+    return x0 <= x1 && y0 <= y1;
+}
+
+// Tile that owns a Gaussian in the backward pass: the tile of its window
+// centre clamped to the grid (always one of the tiles its window touches).
+__device__ __forceinline__ int home_tile(int cx, int cy, const Geom &g) {
+    const int hx = min(max(cx, 0), g.W - 1) >> 4;
+    const int hy = min(max(cy, 0), g.H - 1) >> 4;
+    return hy * g.TX + hx;
+}
+
 // 2^x on the MUFU unit (flush-to-zero for results below the normal range).
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+__device__ __forceinline__ unsigned dynamic_smem_bytes() {
+    unsigned n;
+    asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(n));
+    return n;
 }
 
 __device__ __forceinline__ unsigned lanemask_lt() {
@@ -82,15 +146,41 @@ __device__ __forceinline__ unsigned lanemask_lt() {
     return m;
 }
 
+// Exclusive prefix over the block of one int per thread (any blockDim that is
+// a multiple of 32, at most 1024); `total` gets the block sum.  warp_tot needs
+// blockDim / 32 ints of shared memory.  Called by the whole block.
+__device__ __forceinline__ int block_excl_scan(int v, int *warp_tot, int &total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += u;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    int before = 0;
+    total = 0;
+    for (int w = 0; w < nw; ++w) {
+        const int c = warp_tot[w];
+        before += w < warp ? c : 0;
+        total += c;
+    }
+    __syncthreads();
+    return before + incl - v;
+}
+
 // Launchers (each returns the launch error, cudaSuccess otherwise).
 cudaError_t launch_bin(const float *params, const Geom &g, const Workspace &ws,
                        cudaStream_t s);
+// bin_inside: bin and render in one launch (g.cluster_fwd frames only).
 cudaError_t launch_fwd(const float *params, const Geom &g, const Workspace &ws,
-                       float *image, cudaStream_t s);
+                       float *image, cudaStream_t s, bool bin_inside);
 cudaError_t launch_bwd(const float *params, const float *grad_image, const Geom &g,
                        const Workspace &ws, float *grad_params, cudaStream_t s);
 
 // Dynamic shared memory needed by the kernels for these sizes.
+size_t bin_frame_smem(const Geom &g);
 size_t bin_count_smem(const Geom &g);
 size_t bin_scatter_smem(const Geom &g);
 size_t bwd_smem(const Geom &g);

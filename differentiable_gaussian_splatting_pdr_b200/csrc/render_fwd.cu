@@ -1,30 +1,43 @@
-// Forward tile kernel: I_c(p) = sum_i a_ic * 2^{-(uhat_1^2 + uhat_2^2)} over
+// Forward tile kernels: I_c(p) = sum_i a_ic * 2^{-(uhat_1^2 + uhat_2^2)} over
 // the Gaussians whose k x k window contains p (paper abstract: 5 + C
 // parameters, arbitrary C; reading notes, "Method": additive accumulation).
 //
-// One 128-thread block per (frame, 16x16 tile).  The tile is cut into sixteen
-// 4x4 regions, one per group of 8 lanes; each lane owns a horizontal pixel
-// pair and keeps all C channels of both pixels in registers.  Per batch of
-// the tile's list (ascending Gaussian id):
-//   1. stage: each entry's record is gathered from the per-Gaussian records
-//      and rebased to the tile origin (uhat_j = alpha_j x + beta_j y + K_j in
-//      tile-local pixels), with the window as a 16-bit column mask and a
-//      16-bit row mask;
-//   2. sub-lists: each warp compacts, in list order, the entries whose window
-//      meets each of its four regions, together with the 16-bit mask of the
-//      region's pixels inside the window (ballot + popcount);
-//   3. evaluate: every group walks only its own sub-list, so lanes spend
-//      their issue slots on pixels that can be inside a window.
+// A block renders one 16x16 tile.  The tile is cut into sixteen 4x4 regions,
+// one per group of 16 / PL lanes; a lane owns PL pixels of one row of its
+// region and keeps all C channels of them in registers (PL = 4: 64-thread
+// blocks for large grids; PL = 2: 128-thread blocks, shorter per-lane work,
+// for small grids).  Per batch of the tile's entries (ascending id):
+//   1. stage: each entry's record is rebased to the tile origin
+//      (uhat_j = alpha_j x + beta_j y + K_j in tile-local pixels), with the
+//      window as a 16-bit column mask and a 16-bit row mask;
+//   2. sub-lists: each warp compacts, in entry order, the entries whose
+//      window meets each of its regions, with the 16-bit mask of the region's
+//      pixels inside the window (ballot + popcount);
+//   3. evaluate: every group walks only its own sub-list; a lane evaluates
+//      its pixels from one rebased record, stepping uhat along the row.
 // The per-pixel sum order is the list order: fixed, so results are bitwise
-// reproducible.  Stores are float2 (pixel pairs), coalesced along rows.
+// reproducible.
+//
+// k_fwd reads the tile lists the binner left in the workspace.  For frames of
+// at most kClusterTiles tiles, k_fwd_cluster bins and renders in one launch:
+// one thread-block cluster per frame, block q owning tile q and the q-th
+// chunk of the frame's Gaussians.  Each block counts its chunk per tile; the
+// counts are exchanged through distributed shared memory; each block writes
+// its chunk's entries (stable ranks, as in the binner) into the global list
+// for the backward pass and straight into the list of the owning block's
+// shared memory; then every block renders its tile from its own list.
+#include <cooperative_groups.h>
+
 #include "common.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace pdr {
 
 namespace {
 
-constexpr int kFwdThreads = 128;
-constexpr int kFwdBatch = 128;  // list entries staged per batch
+constexpr int kFwdBatch = 64;          // entries staged per batch (byte offsets fit 16 bits)
+constexpr int kClusterListCap = 1024;  // tile-list entries a clustered block keeps on chip
 
 template <int C>
 struct FwdRec {
@@ -32,46 +45,46 @@ struct FwdRec {
     static constexpr int kVec = (kFloats + 3) / 4;  // float4 per record
 };
 
+template <int PL>
+struct FwdLayout {
+    static constexpr int kThreads = 256 / PL;          // one lane per PL pixels of the tile
+    static constexpr int kLanes = 16 / PL;             // lanes per 4x4 region
+};
+
+// Shared-memory buffers of one rendering block.
 template <int C>
-__global__ void __launch_bounds__(kFwdThreads) k_fwd(const float *__restrict__ params,
-                                                     Geom g,
-                                                     const float4 *__restrict__ gr,
-                                                     const int *__restrict__ offs,
-                                                     const int *__restrict__ ids,
-                                                     float *__restrict__ image,
-                                                     int *__restrict__ err) {
+struct FwdSmem {
+    float4 rec[kFwdBatch * FwdRec<C>::kVec];
+    unsigned win[kFwdBatch];  // window as column bits | row bits << 16 (tile pixels)
+    unsigned sub[16][kFwdBatch];
+    int subn[16];
+};
+
+// Render the entries list[0 .. L) (frame-local ids, ascending) of the tile at
+// (X0, Y0) of frame b into acc.  Called by the whole block.
+template <int C, int PL>
+__device__ __forceinline__ void render_list(const float *__restrict__ params, const Geom &g,
+                                            const float4 *__restrict__ gr, const int *list,
+                                            int L, int b, int X0, int Y0, int *err,
+                                            FwdSmem<C> &S, float (&acc)[PL][C]) {
+    using LY = FwdLayout<PL>;
     constexpr int RV = FwdRec<C>::kVec;
-    __shared__ float4 rec[kFwdBatch * RV];
-    __shared__ unsigned win[kFwdBatch];
-    __shared__ unsigned sub[16][kFwdBatch];
-    __shared__ int subn[16];
-
-    const int b = blockIdx.x / g.T, t = blockIdx.x - b * g.T;
-    const int ty = t / g.TX, tx = t - ty * g.TX;
-    const int X0 = tx * kTile, Y0 = ty * kTile;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int grp = tid >> 3, lig = tid & 7;
-    const int gx = grp & 3;                     // region column; region row == warp
-    const int li = lig & 1, lj = lig >> 1;
-    const int lx = 4 * gx + 2 * li, ly = 4 * warp + lj;  // pixel pair (lx, ly), (lx + 1, ly)
-    const float fx = (float)lx, fy = (float)ly;
-    const unsigned bitA = 1u << (16 + 4 * lj + 2 * li), bitB = bitA << 1;
+    const int grp = tid / LY::kLanes, lig = tid % LY::kLanes;
+    const int gx = grp & 3, gy = grp >> 2;
+    const int lrow = lig / (4 / PL), lcol = (lig % (4 / PL)) * PL;  // lane's row / first column
+    const float fx = (float)(4 * gx + lcol), fy = (float)(4 * gy + lrow);
+    const int bitshift = 16 + 4 * lrow + lcol;  // this lane's bits of a packed sub-list entry
+
     const unsigned lt = lanemask_lt();
-
-    float accA[C], accB[C];
-#pragma unroll
-    for (int c = 0; c < C; ++c) accA[c] = accB[c] = 0.0f;
-
-    int L0, L1;
-    list_range(offs, g, b, t, err, L0, L1);
-    for (int e0 = L0; e0 < L1; e0 += kFwdBatch) {
-        const int n = min(kFwdBatch, L1 - e0);
+    for (int e0 = 0; e0 < L; e0 += kFwdBatch) {
+        const int n = min(kFwdBatch, L - e0);
         __syncthreads();  // the previous batch is fully consumed
-        for (int e = tid; e < n; e += kFwdThreads) {
-            const int i = ids[e0 + e];
+        for (int e = tid; e < n; e += LY::kThreads) {
+            const int i = list[e0 + e];
             if ((unsigned)i >= (unsigned)g.N) {  // never for consistent bins
                 atomicOr(err, kErrBadId);
-                win[e] = 0u;
+                S.win[e] = 0u;
                 continue;
             }
             const size_t gid = (size_t)b * g.N + i;
@@ -93,97 +106,304 @@ __global__ void __launch_bounds__(kFwdThreads) k_fwd(const float *__restrict__ p
             for (int c = 6 + C; c < RV * 4; ++c) r[c] = 0.0f;
 #pragma unroll
             for (int v = 0; v < RV; ++v)
-                rec[e * RV + v] = make_float4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
-            win[e] = (cm & 0xffffu) | ((rm & 0xffffu) << 16);
+                S.rec[e * RV + v] = make_float4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+            // An entry whose window misses the tile (only possible with stale
+            // bins) contributes nothing.
+            S.win[e] = (lx0 <= lx1 && ly0 <= ly1) ? (cm & 0xffffu) | ((rm & 0xffffu) << 16) : 0u;
         }
         __syncthreads();
         {
-            // Sub-lists of this warp's four regions (rows 4*warp .. 4*warp+3).
-            int cnt[4] = {0, 0, 0, 0};
+            // Sub-lists of this warp's regions (region rows ROWS * warp ..).
+            constexpr int RPW = 32 / LY::kLanes;  // regions per warp
+            constexpr int ROWS = RPW / 4;         // region rows per warp
+            int cnt[RPW];
+#pragma unroll
+            for (int q = 0; q < RPW; ++q) cnt[q] = 0;
             const int nr = (n + 31) & ~31;
             for (int e = lane; e < nr; e += 32) {
-                const unsigned wm = e < n ? win[e] : 0u;
-                const unsigned rb = (wm >> (16 + 4 * warp)) & 0xfu;
-                unsigned rs = (rb & 1u) | ((rb & 2u) << 3) | ((rb & 4u) << 6) | ((rb & 8u) << 9);
-                rs *= 0xfu;  // one full nibble per window row of the region
+                const unsigned wm = e < n ? S.win[e] : 0u;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const unsigned cb = (wm >> (4 * q)) & 0xfu;
-                    const unsigned pm = (cb * 0x1111u) & rs;
-                    const unsigned bal = __ballot_sync(0xffffffffu, pm != 0u);
-                    if (pm) sub[4 * warp + q][cnt[q] + __popc(bal & lt)] = (pm << 16) | (unsigned)e;
-                    cnt[q] += __popc(bal);
+                for (int h = 0; h < ROWS; ++h) {
+                    const int row = ROWS * warp + h;
+                    const unsigned rb = (wm >> (16 + 4 * row)) & 0xfu;
+                    unsigned rs = (rb & 1u) | ((rb & 2u) << 3) | ((rb & 4u) << 6) | ((rb & 8u) << 9);
+                    rs *= 0xfu;  // one full nibble per window row of the region
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const unsigned cb = (wm >> (4 * q)) & 0xfu;
+                        const unsigned pm = (cb * 0x1111u) & rs;
+                        const unsigned bal = __ballot_sync(0xffffffffu, pm != 0u);
+                        if (pm)  // pixel mask | byte offset of the entry's record
+                            S.sub[4 * row + q][cnt[4 * h + q] + __popc(bal & lt)] =
+                                (pm << 16) | (unsigned)(e * RV * 16);
+                        cnt[4 * h + q] += __popc(bal);
+                    }
                 }
             }
             if (lane == 0) {
 #pragma unroll
-                for (int q = 0; q < 4; ++q) subn[4 * warp + q] = cnt[q];
+                for (int q = 0; q < RPW; ++q) S.subn[RPW * warp + q] = cnt[q];
             }
         }
         __syncthreads();
-        const int ns = subn[grp];
-        const unsigned *sl = sub[grp];
+        const int ns = S.subn[grp];
+        const unsigned *sl = S.sub[grp];
         for (int s = 0; s < ns; ++s) {
             const unsigned pk = sl[s];
-            const float4 *r4 = rec + (pk & 0xffffu) * RV;
+            const float4 *r4 = reinterpret_cast<const float4 *>(
+                reinterpret_cast<const char *>(S.rec) + (pk & 0xffffu));
             float rr[RV * 4];
 #pragma unroll
             for (int v = 0; v < RV; ++v) {
                 const float4 q = r4[v];
                 rr[4 * v] = q.x; rr[4 * v + 1] = q.y; rr[4 * v + 2] = q.z; rr[4 * v + 3] = q.w;
             }
-            const float uA1 = fmaf(rr[0], fx, fmaf(rr[1], fy, rr[2]));
-            const float uA2 = fmaf(rr[3], fx, fmaf(rr[4], fy, rr[5]));
-            const float uB1 = uA1 + rr[0], uB2 = uA2 + rr[3];
-            const float wA = ex2(fmaf(-uA1, uA1, -uA2 * uA2));
-            const float wB = ex2(fmaf(-uB1, uB1, -uB2 * uB2));
-            if (pk & bitA) {
+            const unsigned bits = pk >> bitshift;
+            float u1 = fmaf(rr[0], fx, fmaf(rr[1], fy, rr[2]));
+            float u2 = fmaf(rr[3], fx, fmaf(rr[4], fy, rr[5]));
 #pragma unroll
-                for (int c = 0; c < C; ++c) accA[c] = fmaf(rr[6 + c], wA, accA[c]);
-            }
-            if (pk & bitB) {
+            for (int j = 0; j < PL; ++j) {
+                if (j) {
+                    u1 += rr[0];
+                    u2 += rr[3];
+                }
+                const float w = ex2(fmaf(-u1, u1, -u2 * u2));
+                if (bits & (1u << j)) {
 #pragma unroll
-                for (int c = 0; c < C; ++c) accB[c] = fmaf(rr[6 + c], wB, accB[c]);
-            }
-        }
-    }
-
-    const int x = X0 + lx, y = Y0 + ly;
-    if (y < g.H && x < g.W) {
-        const bool pair = (x + 1 < g.W) && g.out_vec2;
-#pragma unroll
-        for (int c = 0; c < C; ++c) {
-            float *dst = image + (((size_t)b * C + c) * g.H + y) * g.W + x;
-            if (pair) {
-                *reinterpret_cast<float2 *>(dst) = make_float2(accA[c], accB[c]);
-            } else {
-                dst[0] = accA[c];
-                if (x + 1 < g.W) dst[1] = accB[c];
+                    for (int c = 0; c < C; ++c) acc[j][c] = fmaf(rr[6 + c], w, acc[j][c]);
+                }
             }
         }
     }
 }
 
+template <int C, int PL>
+__device__ __forceinline__ void store_tile(const Geom &g, int b, int X0, int Y0,
+                                           float *__restrict__ image, const float (&acc)[PL][C]) {
+    using LY = FwdLayout<PL>;
+    const int tid = threadIdx.x;
+    const int grp = tid / LY::kLanes, lig = tid % LY::kLanes;
+    const int lrow = lig / (4 / PL), lcol = (lig % (4 / PL)) * PL;
+    const int x = X0 + 4 * (grp & 3) + lcol, y = Y0 + 4 * (grp >> 2) + lrow;
+    if (y >= g.H) return;
+    const bool vec = (x + PL - 1 < g.W) && (PL == 4 ? g.out_vec4 : g.out_vec2);
+#pragma unroll
+    for (int c = 0; c < C; ++c) {
+        float *dst = image + (((size_t)b * C + c) * g.H + y) * g.W + x;
+        if (vec) {
+            if constexpr (PL == 4)
+                *reinterpret_cast<float4 *>(dst) = make_float4(acc[0][c], acc[1][c], acc[2][c], acc[3][c]);
+            else
+                *reinterpret_cast<float2 *>(dst) = make_float2(acc[0][c], acc[1][c]);
+        } else {
+#pragma unroll
+            for (int j = 0; j < PL; ++j)
+                if (x + j < g.W) dst[j] = acc[j][c];
+        }
+    }
+}
+
+template <int C, int PL>
+__global__ void __launch_bounds__(FwdLayout<PL>::kThreads) k_fwd(const float *__restrict__ params,
+                                                                 Geom g,
+                                                                 const float4 *__restrict__ gr,
+                                                                 const int *__restrict__ offs,
+                                                                 const int *__restrict__ ids,
+                                                                 float *__restrict__ image,
+                                                                 int *__restrict__ err) {
+    __shared__ FwdSmem<C> S;
+    const int b = blockIdx.x / g.T, t = blockIdx.x - b * g.T;
+    const int ty = t / g.TX, tx = t - ty * g.TX;
+    const int X0 = tx * kTile, Y0 = ty * kTile;
+    float acc[PL][C];
+#pragma unroll
+    for (int j = 0; j < PL; ++j)
+#pragma unroll
+        for (int c = 0; c < C; ++c) acc[j][c] = 0.0f;
+    int L0, L1;
+    list_range(offs, g, b, t, err, L0, L1);
+    render_list<C, PL>(params, g, gr, ids + L0, L1 - L0, b, X0, Y0, err, S, acc);
+    store_tile<C, PL>(g, b, X0, Y0, image, acc);
+}
+
+// Bins and renders one small frame per thread-block cluster (grid (T, B),
+// cluster (T, 1, 1)); block q = tile q owns the Gaussians [q * chunk, ...).
+template <int C, int PL>
+__global__ void __launch_bounds__(FwdLayout<PL>::kThreads) k_fwd_cluster(
+    const float *__restrict__ params, Geom g, float4 *__restrict__ gr, int *__restrict__ offs,
+    int *__restrict__ ids, float *__restrict__ image, int *__restrict__ err) {
+    constexpr int NT = FwdLayout<PL>::kThreads;
+    constexpr int NW = NT / 32;
+    __shared__ FwdSmem<C> S;
+    __shared__ int cnt[kClusterTiles];                 // this chunk's count per tile
+    __shared__ int tab[kClusterTiles][kClusterTiles];  // tab[r][t] = count of chunk r in tile t
+    __shared__ int base[kClusterTiles];                // next list slot of this chunk, per tile
+    __shared__ int tstart[kClusterTiles + 1];          // frame's tile offsets (relative)
+    __shared__ unsigned masks[NW][kClusterTiles];
+    __shared__ int list[kClusterListCap];              // this tile's entries, filled by the cluster
+
+    cg::cluster_group cluster = cg::this_cluster();
+    const int T = g.T;
+    const int q = (int)cluster.block_rank();  // == tile index
+    const int b = blockIdx.y;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const unsigned lt = lanemask_lt();
+    if (b == 0 && q == 0 && tid == 0) *err = 0;
+    if (tid < kClusterTiles) cnt[tid] = 0;
+    if (tid < NW * kClusterTiles) masks[tid / kClusterTiles][tid % kClusterTiles] = 0u;
+    __syncthreads();
+
+    // 1. records and per-tile counts of this block's chunk
+    const int chunk = (g.N + T - 1) / T;
+    const int i0 = min(q * chunk, g.N), i1 = min(i0 + chunk, g.N);
+    for (int i = i0 + tid; i < i1; i += NT) {
+        const size_t gid = (size_t)b * g.N + i;
+        float4 A, Q;
+        gaussian_record(params + gid * g.P, A, Q);
+        gr[2 * gid] = A;
+        gr[2 * gid + 1] = Q;
+        int x0, x1, y0, y1;
+        if (window_rect(__float_as_int(Q.z), __float_as_int(Q.w), g, x0, x1, y0, y1)) {
+            for (int yy = y0 >> 4; yy <= (y1 >> 4); ++yy)
+                for (int xx = x0 >> 4; xx <= (x1 >> 4); ++xx) atomicAdd(&cnt[yy * g.TX + xx], 1);
+        }
+    }
+    cluster.sync();
+
+    // 2. every block reads all chunks' counts (distributed shared memory)
+    for (int j = tid; j < T * T; j += NT) {
+        const int r = j / T, tt = j - r * T;
+        tab[r][tt] = *cluster.map_shared_rank(cnt + tt, r);
+    }
+    __syncthreads();
+    if (tid == 0) {
+        int run = 0;
+        for (int tt = 0; tt < T; ++tt) {
+            tstart[tt] = run;
+            int below = 0;
+            for (int r = 0; r < T; ++r) {
+                below += r < q ? tab[r][tt] : 0;
+                run += tab[r][tt];
+            }
+            base[tt] = tstart[tt] + below;
+        }
+        tstart[T] = run;
+    }
+    __syncthreads();
+    const int frame0 = b * g.cap;
+    if (q == 0)
+        for (int tt = tid; tt <= T; tt += NT) offs[(size_t)b * (T + 1) + tt] = frame0 + tstart[tt];
+
+    // 3. stable scatter of this chunk: global list + the owning block's list
+    const long long lo = frame0, hi = lo + g.cap;
+    for (int s = i0; s < i1; s += NT) {
+        const int i = s + tid;
+        int tx0 = 1, tx1 = 0, ty0 = 1, ty1 = 0;
+        if (i < i1) {
+            const float4 Q = gr[2 * ((size_t)b * g.N + i) + 1];
+            int x0, x1, y0, y1;
+            if (window_rect(__float_as_int(Q.z), __float_as_int(Q.w), g, x0, x1, y0, y1)) {
+                tx0 = x0 >> 4; tx1 = x1 >> 4; ty0 = y0 >> 4; ty1 = y1 >> 4;
+            }
+        }
+        for (int yy = ty0; yy <= ty1; ++yy)
+            for (int xx = tx0; xx <= tx1; ++xx) atomicOr(&masks[warp][yy * g.TX + xx], 1u << lane);
+        __syncthreads();
+        for (int yy = ty0; yy <= ty1; ++yy)
+            for (int xx = tx0; xx <= tx1; ++xx) {
+                const int tt = yy * g.TX + xx;
+                int pre = base[tt] + __popc(masks[warp][tt] & lt);
+                for (int w = 0; w < warp; ++w) pre += __popc(masks[w][tt]);
+                const long long slot = (long long)frame0 + pre;
+                if (slot >= lo && slot < hi) {
+                    ids[slot] = i;
+                    const int local = pre - tstart[tt];
+                    if (local < kClusterListCap) *cluster.map_shared_rank(list + local, tt) = i;
+                } else {
+                    atomicOr(err, kErrListBounds);
+                }
+            }
+        __syncthreads();
+        if (tid < T) {
+            int add = 0;
+            for (int w = 0; w < NW; ++w) add += __popc(masks[w][tid]);
+            base[tid] += add;
+        }
+        __syncthreads();
+        if (tid < NW * kClusterTiles) masks[tid / kClusterTiles][tid % kClusterTiles] = 0u;
+        __syncthreads();
+    }
+    cluster.sync();  // every list is complete; no block touches another's memory after this
+
+    // 4. render this tile from its own list
+    const int ty = q / g.TX, tx = q - ty * g.TX;
+    const int X0 = tx * kTile, Y0 = ty * kTile;
+    float acc[PL][C];
+#pragma unroll
+    for (int j = 0; j < PL; ++j)
+#pragma unroll
+        for (int c = 0; c < C; ++c) acc[j][c] = 0.0f;
+    const int L = tstart[q + 1] - tstart[q];
+    const int *src = L <= kClusterListCap ? list : ids + frame0 + tstart[q];
+    render_list<C, PL>(params, g, gr, src, L, b, X0, Y0, err, S, acc);
+    store_tile<C, PL>(g, b, X0, Y0, image, acc);
+}
+
+template <int C, int PL>
+cudaError_t launch_fwd_cluster(const float *params, const Geom &g, const Workspace &ws,
+                               float *image, cudaStream_t s) {
+        cudaError_t e;
+        if (g.T > 8) {
+            e = cudaFuncSetAttribute(k_fwd_cluster<C, PL>,
+                                     cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+            if (e != cudaSuccess) return e;
+        }
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        cfg.gridDim = dim3(g.T, g.B, 1);
+        cfg.blockDim = dim3(FwdLayout<PL>::kThreads, 1, 1);
+        cfg.dynamicSmemBytes = 0;
+        cfg.stream = s;
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = g.T;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, k_fwd_cluster<C, PL>, params, g, ws.gr, ws.offs, ws.ids,
+                               image, ws.err);
+        if (e != cudaSuccess) return e;
+        return cudaGetLastError();
+}
+
 template <int C>
-cudaError_t launch_fwd_c(const float *params, const Geom &g, const Workspace &ws,
-                         float *image, cudaStream_t s) {
-    k_fwd<C><<<g.B * g.T, kFwdThreads, 0, s>>>(params, g, ws.gr, ws.offs, ws.ids, image, ws.err);
+cudaError_t launch_fwd_c(const float *params, const Geom &g, const Workspace &ws, float *image,
+                         cudaStream_t s, bool bin_inside) {
+    if (bin_inside)
+        return g.fwd_pl == 2 ? launch_fwd_cluster<C, 2>(params, g, ws, image, s)
+                             : launch_fwd_cluster<C, 4>(params, g, ws, image, s);
+    if (g.fwd_pl == 2)
+        k_fwd<C, 2><<<g.B * g.T, FwdLayout<2>::kThreads, 0, s>>>(params, g, ws.gr, ws.offs,
+                                                                 ws.ids, image, ws.err);
+    else
+        k_fwd<C, 4><<<g.B * g.T, FwdLayout<4>::kThreads, 0, s>>>(params, g, ws.gr, ws.offs,
+                                                                 ws.ids, image, ws.err);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_fwd(const float *params, const Geom &g, const Workspace &ws,
-                       float *image, cudaStream_t s) {
+cudaError_t launch_fwd(const float *params, const Geom &g, const Workspace &ws, float *image,
+                       cudaStream_t s, bool bin_inside) {
     switch (g.C) {
-        case 1: return launch_fwd_c<1>(params, g, ws, image, s);
-        case 2: return launch_fwd_c<2>(params, g, ws, image, s);
-        case 3: return launch_fwd_c<3>(params, g, ws, image, s);
-        case 4: return launch_fwd_c<4>(params, g, ws, image, s);
-        case 5: return launch_fwd_c<5>(params, g, ws, image, s);
-        case 6: return launch_fwd_c<6>(params, g, ws, image, s);
-        case 7: return launch_fwd_c<7>(params, g, ws, image, s);
-        case 8: return launch_fwd_c<8>(params, g, ws, image, s);
+        case 1: return launch_fwd_c<1>(params, g, ws, image, s, bin_inside);
+        case 2: return launch_fwd_c<2>(params, g, ws, image, s, bin_inside);
+        case 3: return launch_fwd_c<3>(params, g, ws, image, s, bin_inside);
+        case 4: return launch_fwd_c<4>(params, g, ws, image, s, bin_inside);
+        case 5: return launch_fwd_c<5>(params, g, ws, image, s, bin_inside);
+        case 6: return launch_fwd_c<6>(params, g, ws, image, s, bin_inside);
+        case 7: return launch_fwd_c<7>(params, g, ws, image, s, bin_inside);
+        case 8: return launch_fwd_c<8>(params, g, ws, image, s, bin_inside);
         default: return cudaErrorInvalidValue;
     }
 }
