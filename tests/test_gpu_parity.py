@@ -132,6 +132,14 @@ def _edge_params(rng, B, N, C, H, W, k, smean=0.4, ssd=0.4):
     (1, 64, 3, 16, 16, 1),      # single-pixel windows
     (4, 1, 4, 20, 30, 5),       # N = 1
     (1, 500, 6, 7, 9, 3),       # grid smaller than a tile
+    # pixel-pair backward (C <= 4, k 13 and 15) and the scalar one beside it, centres on and off the grid
+    (2, 400, 3, 40, 56, 15),    # ragged, both window parities, rows wider than a tile
+    (1, 300, 4, 23, 37, 9),     # ragged both ways, slots kept per lane
+    (2, 200, 1, 33, 47, 11),
+    (1, 100, 2, 50, 20, 13),
+    (1, 250, 1, 37, 29, 15),
+    (3, 80, 3, 16, 16, 3),
+    (2, 120, 4, 30, 45, 7),
 ])
 def test_edge_shapes(B, N, C, H, W, k):
     rng = np.random.default_rng(B * 1000 + N + C)
