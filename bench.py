@@ -84,14 +84,17 @@ def source_hash(*names) -> str:
 KERNEL_SOURCES = {"k_fwd": ("render_fwd.cu", "common.cuh"),
                   "k_fwd_cluster": ("render_fwd.cu", "common.cuh"),
                   "k_bwd": ("render_bwd.cu", "common.cuh")}
-CLUSTER_MAX_TILES = 16   # frames of at most this many tiles bin + render in k_fwd_cluster
+CLUSTER_MAX_TILES = 16       # frames of at most this many tiles ...
+CLUSTER_MAX_BLOCKS = 4 * 148  # ... in launches of at most this many blocks: k_fwd_cluster
 
 
 def forward_kernel(w) -> str:
-    """The forward kernel the library launches for workload w: frames of at
-    most 16 tiles are binned and rendered by one clustered launch."""
+    """The forward kernel the library launches for workload w: small launches
+    of frames of at most 16 tiles are binned and rendered by one clustered
+    launch; everything else is binned first and rendered by k_fwd."""
     tiles = -(-w.H // 16) * -(-w.W // 16)
-    return "k_fwd_cluster" if tiles <= CLUSTER_MAX_TILES else "k_fwd"
+    fused = tiles <= CLUSTER_MAX_TILES and w.B * tiles <= CLUSTER_MAX_BLOCKS
+    return "k_fwd_cluster" if fused else "k_fwd"
 
 
 def aggregate_over_ranks(torch, dist, world, device, evals, step_ms, extra_ms=()):

@@ -52,7 +52,10 @@ pdr_status make_geom(int B, int N, int C, int H, int W, int k, Geom *g) {
     if (ft > 1024) ft = 1024;
     if (B > 148 && ft > 512) ft = 512;  // more frames than SMs: more, smaller blocks
     g->frame_threads = ft;
-    g->cluster_fwd = T <= kClusterTiles;
+    // Bins + render in one clustered launch only while the launch is small
+    // (latency-bound); larger batches of small frames run faster as separate
+    // binning and render launches (measured on B200).
+    g->cluster_fwd = T <= kClusterTiles && (long long)B * T <= kClusterMaxBlocks;
     g->fwd_pl = (long long)B * T <= 2368 ? 2 : 4;  // small grids: more, shorter lanes per tile
     g->out_vec2 = 0;
     g->out_vec4 = 0;

@@ -41,7 +41,8 @@ struct Geom {
 constexpr int kBinChunk = 1024;        // Gaussians per binning block (large frames)
 constexpr int kFrameBlockMaxT = 256;   // small frames: at most this many tiles
 constexpr int kFrameBlockMaxN = 16384; // and at most this many Gaussians
-constexpr int kClusterTiles = 16;      // frames up to this many tiles: one cluster per frame
+constexpr int kClusterTiles = 16;            // frames up to this many tiles: one cluster per frame
+constexpr int kClusterMaxBlocks = 4 * 148;   // ... while the launch has at most this many blocks
 
 // Per-Gaussian record written by the binner and read by both render kernels
 // (two float4 per Gaussian, 32 bytes):

@@ -38,6 +38,7 @@ namespace {
 
 constexpr int kFwdBatch = 64;          // entries staged per batch (byte offsets fit 16 bits)
 constexpr int kClusterListCap = 1024;  // tile-list entries a clustered block keeps on chip
+constexpr int kChunkSmem = 256;        // Gaussians per clustered block whose records stay on chip
 
 template <int C>
 struct FwdRec {
@@ -62,10 +63,11 @@ struct FwdSmem {
 
 // Render the entries list[0 .. L) (frame-local ids, ascending) of the tile at
 // (X0, Y0) of frame b into acc.  Called by the whole block.
-template <int C, int PL>
-__device__ __forceinline__ void render_list(const float *__restrict__ params, const Geom &g,
-                                            const float4 *__restrict__ gr, const int *list,
-                                            int L, int b, int X0, int Y0, int *err,
+// fetch(i, A, Q, amp) supplies the record and amplitudes of frame-local
+// Gaussian i (from global memory, or from a cluster peer's shared memory).
+template <int C, int PL, typename Fetch>
+__device__ __forceinline__ void render_list(const Geom &g, Fetch fetch, const int *list,
+                                            int L, int X0, int Y0, int *err,
                                             FwdSmem<C> &S, float (&acc)[PL][C]) {
     using LY = FwdLayout<PL>;
     constexpr int RV = FwdRec<C>::kVec;
@@ -87,8 +89,9 @@ __device__ __forceinline__ void render_list(const float *__restrict__ params, co
                 S.win[e] = 0u;
                 continue;
             }
-            const size_t gid = (size_t)b * g.N + i;
-            const float4 A = gr[2 * gid], Q = gr[2 * gid + 1];
+            float4 A, Q;
+            float amp[C];
+            fetch(i, A, Q, amp);
             const float mx = A.x - (float)X0, my = A.y - (float)Y0;
             const float K1 = -fmaf(A.z, mx, A.w * my);
             const float K2 = -fmaf(Q.x, mx, Q.y * my);
@@ -99,9 +102,8 @@ __device__ __forceinline__ void render_list(const float *__restrict__ params, co
             const unsigned rm = (2u << ly1) - (1u << ly0);
             float r[RV * 4];
             r[0] = A.z; r[1] = A.w; r[2] = K1; r[3] = Q.x; r[4] = Q.y; r[5] = K2;
-            const float *pa = params + gid * g.P + 5;
 #pragma unroll
-            for (int c = 0; c < C; ++c) r[6 + c] = pa[c];
+            for (int c = 0; c < C; ++c) r[6 + c] = amp[c];
 #pragma unroll
             for (int c = 6 + C; c < RV * 4; ++c) r[c] = 0.0f;
 #pragma unroll
@@ -222,7 +224,15 @@ __global__ void __launch_bounds__(FwdLayout<PL>::kThreads) k_fwd(const float *__
         for (int c = 0; c < C; ++c) acc[j][c] = 0.0f;
     int L0, L1;
     list_range(offs, g, b, t, err, L0, L1);
-    render_list<C, PL>(params, g, gr, ids + L0, L1 - L0, b, X0, Y0, err, S, acc);
+    auto fetch = [&](int i, float4 &A, float4 &Q, float (&amp)[C]) {
+        const size_t gid = (size_t)b * g.N + i;
+        A = gr[2 * gid];
+        Q = gr[2 * gid + 1];
+        const float *pa = params + gid * g.P + 5;
+#pragma unroll
+        for (int c = 0; c < C; ++c) amp[c] = pa[c];
+    };
+    render_list<C, PL>(g, fetch, ids + L0, L1 - L0, X0, Y0, err, S, acc);
     store_tile<C, PL>(g, b, X0, Y0, image, acc);
 }
 
@@ -241,6 +251,8 @@ __global__ void __launch_bounds__(FwdLayout<PL>::kThreads) k_fwd_cluster(
     __shared__ int tstart[kClusterTiles + 1];          // frame's tile offsets (relative)
     __shared__ unsigned masks[NW][kClusterTiles];
     __shared__ int list[kClusterListCap];              // this tile's entries, filled by the cluster
+    __shared__ float4 crec[kChunkSmem][2];             // this chunk's records (read by the cluster)
+    __shared__ float camp[kChunkSmem][C];              // and amplitudes
 
     cg::cluster_group cluster = cg::this_cluster();
     const int T = g.T;
@@ -255,6 +267,7 @@ __global__ void __launch_bounds__(FwdLayout<PL>::kThreads) k_fwd_cluster(
 
     // 1. records and per-tile counts of this block's chunk
     const int chunk = (g.N + T - 1) / T;
+    const bool onchip = chunk <= kChunkSmem;  // same for every block of the cluster
     const int i0 = min(q * chunk, g.N), i1 = min(i0 + chunk, g.N);
     for (int i = i0 + tid; i < i1; i += NT) {
         const size_t gid = (size_t)b * g.N + i;
@@ -262,6 +275,13 @@ __global__ void __launch_bounds__(FwdLayout<PL>::kThreads) k_fwd_cluster(
         gaussian_record(params + gid * g.P, A, Q);
         gr[2 * gid] = A;
         gr[2 * gid + 1] = Q;
+        if (onchip) {
+            crec[i - i0][0] = A;
+            crec[i - i0][1] = Q;
+            const float *pa = params + gid * g.P + 5;
+#pragma unroll
+            for (int c = 0; c < C; ++c) camp[i - i0][c] = pa[c];
+        }
         int x0, x1, y0, y1;
         if (window_rect(__float_as_int(Q.z), __float_as_int(Q.w), g, x0, x1, y0, y1)) {
             for (int yy = y0 >> 4; yy <= (y1 >> 4); ++yy)
@@ -276,18 +296,26 @@ __global__ void __launch_bounds__(FwdLayout<PL>::kThreads) k_fwd_cluster(
         tab[r][tt] = *cluster.map_shared_rank(cnt + tt, r);
     }
     __syncthreads();
-    if (tid == 0) {
-        int run = 0;
-        for (int tt = 0; tt < T; ++tt) {
-            tstart[tt] = run;
-            int below = 0;
+    if (warp == 0) {  // tile offsets: lane tt sums column tt, then a warp scan over tiles
+        int col = 0, below = 0;
+        if (lane < T) {
             for (int r = 0; r < T; ++r) {
-                below += r < q ? tab[r][tt] : 0;
-                run += tab[r][tt];
+                const int v = tab[r][lane];
+                col += v;
+                below += r < q ? v : 0;
             }
-            base[tt] = tstart[tt] + below;
         }
-        tstart[T] = run;
+        int incl = col;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int u = __shfl_up_sync(0xffffffffu, incl, d);
+            if (lane >= d) incl += u;
+        }
+        if (lane < T) {
+            tstart[lane] = incl - col;
+            base[lane] = incl - col + below;
+        }
+        if (lane == T - 1) tstart[T] = incl;
     }
     __syncthreads();
     const int frame0 = b * g.cap;
@@ -333,7 +361,7 @@ __global__ void __launch_bounds__(FwdLayout<PL>::kThreads) k_fwd_cluster(
         if (tid < NW * kClusterTiles) masks[tid / kClusterTiles][tid % kClusterTiles] = 0u;
         __syncthreads();
     }
-    cluster.sync();  // every list is complete; no block touches another's memory after this
+    cluster.sync();  // every list is complete; only the records are read across blocks after this
 
     // 4. render this tile from its own list
     const int ty = q / g.TX, tx = q - ty * g.TX;
@@ -345,8 +373,31 @@ __global__ void __launch_bounds__(FwdLayout<PL>::kThreads) k_fwd_cluster(
         for (int c = 0; c < C; ++c) acc[j][c] = 0.0f;
     const int L = tstart[q + 1] - tstart[q];
     const int *src = L <= kClusterListCap ? list : ids + frame0 + tstart[q];
-    render_list<C, PL>(params, g, gr, src, L, b, X0, Y0, err, S, acc);
+    if (onchip) {
+        // Records from the chunk owners' shared memory (distributed shared memory).
+        auto fetch = [&](int i, float4 &A, float4 &Q, float (&amp)[C]) {
+            const int r = i / chunk, li = i - r * chunk;
+            const float4 *pr = cluster.map_shared_rank(&crec[li][0], r);
+            const float *pa = cluster.map_shared_rank(&camp[li][0], r);
+            A = pr[0];
+            Q = pr[1];
+#pragma unroll
+            for (int c = 0; c < C; ++c) amp[c] = pa[c];
+        };
+        render_list<C, PL>(g, fetch, src, L, X0, Y0, err, S, acc);
+    } else {
+        auto fetch = [&](int i, float4 &A, float4 &Q, float (&amp)[C]) {
+            const size_t gid = (size_t)b * g.N + i;
+            A = gr[2 * gid];
+            Q = gr[2 * gid + 1];
+            const float *pa = params + gid * g.P + 5;
+#pragma unroll
+            for (int c = 0; c < C; ++c) amp[c] = pa[c];
+        };
+        render_list<C, PL>(g, fetch, src, L, X0, Y0, err, S, acc);
+    }
     store_tile<C, PL>(g, b, X0, Y0, image, acc);
+    if (onchip) cluster.sync();  // peers may still read this block's records
 }
 
 template <int C, int PL>

@@ -87,7 +87,8 @@ def test_single_rank_aggregate_is_identity():
 def test_forward_kernel_attribution():
     assert bench.forward_kernel(WORKLOADS["mono64"]) == "k_fwd_cluster"   # 16 tiles
     assert bench.forward_kernel(WORKLOADS["rgb128"]) == "k_fwd"           # 64 tiles
-    assert bench.forward_kernel(WORKLOADS["field32x64"]) == "k_fwd_cluster"
+    assert bench.forward_kernel(WORKLOADS["field32x64"]) == "k_fwd"            # 2560 blocks
+    assert bench.forward_kernel(WORKLOADS["tiny"]) == "k_fwd_cluster"
 
 
 @pytest.mark.slow
