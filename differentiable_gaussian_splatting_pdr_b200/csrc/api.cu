@@ -50,7 +50,10 @@ pdr_status make_geom(int B, int N, int C, int H, int W, int k, Geom *g) {
     g->frame_block = T <= kFrameBlockMaxT && N <= kFrameBlockMaxN;
     int ft = ((N + 31) / 32) * 32;
     if (ft > 1024) ft = 1024;
-    if (B > 148 && ft > 512) ft = 512;  // more frames than SMs: more, smaller blocks
+    // More frames than SMs: smaller blocks, so that all frames are resident in
+    // one wave (about 1024 binning threads per SM).
+    const long long per_sm = ((long long)B + 147) / 148;
+    while (ft > 128 && per_sm * ft > 1024) ft = ((ft / 2 + 31) / 32) * 32;
     g->frame_threads = ft;
     // Bins + render in one clustered launch only while the launch is small
     // (latency-bound); larger batches of small frames run faster as separate

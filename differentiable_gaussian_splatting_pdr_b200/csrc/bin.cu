@@ -9,12 +9,12 @@
 //             per-Gaussian record (window centre, rotated and scaled axes)
 //             and the chunk's per-tile counts (integer shared-memory atomics
 //             count only; they never decide a position);
-//   k_scan    one block per frame, one thread per tile: exclusive prefix of
-//             the tile's counts over the chunks (loads issued in independent
-//             batches), then a block scan of the tile totals gives each tile
-//             its list start;
+//   k_scan_tiles / k_scan_frames
+//             exclusive prefix of each tile's counts over the chunks (32 tiles
+//             x 32 chunks per step through shared memory), then one block per
+//             frame scans the tile totals into the tiles' list starts;
 //   k_scatter one block per (frame, chunk): stable ranks in rounds of
-//             blockDim Gaussians -- rank in a tile = earlier chunks (k_scan) +
+//             blockDim Gaussians -- rank in a tile = earlier chunks (the scans) +
 //             earlier rounds + earlier warps' popcounts + lanes below in this
 //             warp (per-warp lane bitmasks) -- so positions never depend on
 //             the order in which atomics land.
@@ -29,7 +29,6 @@ namespace pdr {
 namespace {
 
 constexpr int kCountThreads = 256;
-constexpr int kScanBatch = 8;
 
 __global__ void __launch_bounds__(kCountThreads) k_count(const float *__restrict__ params,
                                                          Geom g, float4 *__restrict__ gr,
@@ -94,37 +93,60 @@ __device__ __forceinline__ int block_incl_scan(int v, int *warp_tot, int &total)
 }
 
 // hist[b][c][t] <- exclusive prefix over c of the counts (relative to the
-// tile's list start); offs[b][t] <- the tile's absolute list start.
-__global__ void __launch_bounds__(1024) k_scan(Geom g, int *__restrict__ hist,
-                                               int *__restrict__ offs) {
+// tile's list start); offs[b][t] <- the tile's total (turned into the
+// absolute list start by k_scan_frames).  Block (x, b) takes tiles
+// 32x .. 32x + 31 of frame b: the chunk counts pass through shared memory
+// 32 chunks at a time (coalesced along the tiles on both sides), and warp w
+// scans tile 32x + w over those chunks, carrying the running sum.
+__global__ void __launch_bounds__(1024) k_scan_tiles(Geom g, int *__restrict__ hist,
+                                                     int *__restrict__ offs) {
+    __shared__ int v[32][33];  // [chunk][tile], padded against bank conflicts
+    const int b = blockIdx.y, t0 = blockIdx.x * 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int *h = hist + (size_t)b * g.nchunks * g.T;
+    int carry = 0;  // warp's tile: sum of the chunks already scanned
+    for (int c0 = 0; c0 < g.nchunks; c0 += 32) {
+        {
+            const int c = c0 + warp, t = t0 + lane;  // load: warp = chunk, lane = tile
+            v[warp][lane] = (c < g.nchunks && t < g.T) ? h[(size_t)c * g.T + t] : 0;
+        }
+        __syncthreads();
+        {
+            const int x = v[lane][warp];  // scan: warp = tile, lane = chunk
+            int incl = x;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const int u = __shfl_up_sync(0xffffffffu, incl, d);
+                if (lane >= d) incl += u;
+            }
+            v[lane][warp] = carry + incl - x;
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        __syncthreads();
+        {
+            const int c = c0 + warp, t = t0 + lane;
+            if (c < g.nchunks && t < g.T) h[(size_t)c * g.T + t] = v[warp][lane];
+        }
+        __syncthreads();
+    }
+    if (lane == 0 && t0 + warp < g.T) offs[(size_t)b * (g.T + 1) + t0 + warp] = carry;
+}
+
+// offs[b][t] <- frame start + exclusive prefix over the tiles of their totals.
+__global__ void __launch_bounds__(1024) k_scan_frames(Geom g, int *__restrict__ offs) {
     __shared__ int warp_tot[32];
     const int b = blockIdx.x;
-    const int frame_base = b * g.cap;
-    const size_t stride = g.T;
-    int carry = 0;
+    int *o = offs + (size_t)b * (g.T + 1);
+    int carry = b * g.cap;
     for (int t0 = 0; t0 < g.T; t0 += blockDim.x) {
         const int t = t0 + threadIdx.x;
-        int tot = 0;
-        if (t < g.T) {
-            int *h = hist + (size_t)b * g.nchunks * stride + t;
-            for (int c0 = 0; c0 < g.nchunks; c0 += kScanBatch) {
-                int v[kScanBatch];
-#pragma unroll
-                for (int j = 0; j < kScanBatch; ++j)
-                    v[j] = c0 + j < g.nchunks ? h[(c0 + j) * stride] : 0;
-#pragma unroll
-                for (int j = 0; j < kScanBatch; ++j) {
-                    if (c0 + j < g.nchunks) h[(c0 + j) * stride] = tot;
-                    tot += v[j];
-                }
-            }
-        }
+        const int tot = t < g.T ? o[t] : 0;
         int total;
         const int incl = block_incl_scan(tot, warp_tot, total);
-        if (t < g.T) offs[(size_t)b * (g.T + 1) + t] = frame_base + carry + incl - tot;
+        if (t < g.T) o[t] = carry + incl - tot;
         carry += total;
     }
-    if (threadIdx.x == 0) offs[(size_t)b * (g.T + 1) + g.T] = frame_base + carry;
+    if (threadIdx.x == 0) o[g.T] = carry;
 }
 
 __global__ void k_scatter(Geom g, const float4 *__restrict__ gr, const int *__restrict__ hist,
@@ -331,7 +353,8 @@ cudaError_t launch_bin(const float *params, const Geom &g, const Workspace &ws,
     const dim3 grid(g.nchunks, g.B);
     const int scan_threads = g.T >= 1024 ? 1024 : ((g.T + 31) / 32) * 32;
     k_count<<<grid, kCountThreads, sc, s>>>(params, g, ws.gr, ws.hist, ws.err);
-    k_scan<<<g.B, scan_threads, 0, s>>>(g, ws.hist, ws.offs);
+    k_scan_tiles<<<dim3((g.T + 31) / 32, g.B), 1024, 0, s>>>(g, ws.hist, ws.offs);
+    k_scan_frames<<<g.B, scan_threads, 0, s>>>(g, ws.offs);
     k_scatter<<<grid, 32 * g.scatter_warps, ss, s>>>(g, ws.gr, ws.hist, ws.offs, ws.ids, ws.err);
     return cudaGetLastError();
 }

@@ -221,3 +221,23 @@ def test_separate_bins_then_render_matches_one_call():
     img2, dp2 = run_gpu(p, g, w.H, w.W, w.k)
     assert np.array_equal(img.cpu().numpy(), img2)
     assert np.array_equal(dp.cpu().numpy(), dp2)
+
+
+@pytest.mark.parametrize("B,N,C,H,W,k", [
+    (2, 40000, 1, 112, 144, 5),   # large frames: chunked count, two scan passes, 63 tiles
+    (1, 20000, 2, 300, 240, 3),   # 285 tiles (more than one frame block takes), 20 chunks
+])
+def test_chunked_binning_paths(B, N, C, H, W, k):
+    """Frames too large for one binning block (count, two-level scan, scatter)."""
+    rng = np.random.default_rng(N + H)
+    p = _edge_params(rng, B, N, C, H, W, k, smean=0.2, ssd=0.3)
+    g = rng.standard_normal((B, C, H, W)).astype(np.float32)
+    check_all(p, g, H, W, k)
+
+
+@pytest.mark.parametrize("B", [149, 300, 450])
+def test_many_small_frames(B):
+    """More frames than SMs: smaller frame-binning blocks, one wave."""
+    w = WORKLOADS["field32x64"].scaled(B=B, N=300)
+    p, g = make_inputs(w)
+    check_all(p, g, w.H, w.W, w.k)
