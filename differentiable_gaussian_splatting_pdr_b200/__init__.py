@@ -11,7 +11,10 @@ from .api import (  # noqa: F401
     bin_tiles,
     build_bins,
     check_device_error,
+    l1_ssim,
+    l1_ssim_loss,
     list_capacity_per_frame,
+    loss_workspace_bytes,
     render,
     render_bwd,
     render_fwd,

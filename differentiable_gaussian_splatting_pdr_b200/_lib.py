@@ -23,6 +23,8 @@ STATUS_NAMES = {
     6: "PDR_ERR_TOO_LARGE",
 }
 
+STATUS_CODES = {name: code for code, name in STATUS_NAMES.items()}
+
 # Every symbol include/pdr.h declares, with (restype, argtypes).
 _vp, _i, _sz, _ll = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_longlong
 SIGNATURES = {
@@ -37,6 +39,8 @@ SIGNATURES = {
     "pdr_step_host": (_i, [_vp, _vp, _vp, _vp] + [_i] * 6 + [_vp] * 5 + [_sz, _vp]),
     "pdr_check_device_error": (_i, [_vp, _vp]),
     "pdr_render_fwd_noalloc": (_i, [_vp] + [_i] * 6 + [_vp, _vp]),
+    "pdr_loss_workspace_bytes": (_sz, [_i] * 4),
+    "pdr_loss_l1_ssim": (_i, [_vp, _vp] + [_i] * 4 + [ctypes.c_float, ctypes.c_float] + [_vp] * 3 + [_sz, _vp]),
 }
 
 _lib = None

@@ -214,3 +214,54 @@ class _Render(torch.autograd.Function):
 def render(params: torch.Tensor, H: int, W: int, k: int) -> torch.Tensor:
     """Differentiable render: image [B, C, H, W] from params [B, N, 5 + C]."""
     return _Render.apply(params.contiguous(), H, W, k)
+
+
+def loss_workspace_bytes(B: int, C: int, H: int, W: int) -> int:
+    return int(_lib.load().pdr_loss_workspace_bytes(B, C, H, W))
+
+
+def l1_ssim_loss(image: torch.Tensor, target: torch.Tensor, lam: float = 0.2,
+                 data_range: float = 1.0, workspace: torch.Tensor | None = None,
+                 grad_out: torch.Tensor | None = None):
+    """L1 + SSIM training loss and dL/dimage (see pdr_loss_l1_ssim).
+
+    image, target: contiguous fp32 CUDA tensors [B, C, H, W].  Returns
+    (loss, grad): a 1-element device tensor and a tensor like image.  The
+    target receives no gradient."""
+    lib = _lib.load()
+    for t in (image, target):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.float32 \
+                or t.dim() != 4 or not t.is_contiguous():
+            raise ValueError("image and target must be contiguous fp32 CUDA tensors [B, C, H, W]")
+    if image.shape != target.shape:
+        raise ValueError("image and target shapes differ")
+    B, C, H, W = image.shape
+    dev = image.device
+    nb = loss_workspace_bytes(B, C, H, W)
+    if workspace is None or workspace.numel() < nb:
+        workspace = torch.empty(max(nb, 256), dtype=torch.uint8, device=dev)
+    grad = torch.empty_like(image) if grad_out is None else grad_out
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    _lib.check("pdr_loss_l1_ssim", lib.pdr_loss_l1_ssim(
+        _ptr(image), _ptr(target), B, C, H, W, float(lam), float(data_range), _ptr(loss),
+        _ptr(grad), _ptr(workspace), workspace.numel(), _stream(dev)))
+    return loss, grad
+
+
+class _L1Ssim(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, image, target, lam, data_range):
+        loss, grad = l1_ssim_loss(image, target, lam, data_range)
+        ctx.save_for_backward(grad)
+        return loss[0]
+
+    @staticmethod
+    def backward(ctx, g):
+        (grad,) = ctx.saved_tensors
+        return grad * g, None, None, None
+
+
+def l1_ssim(image: torch.Tensor, target: torch.Tensor, lam: float = 0.2,
+            data_range: float = 1.0) -> torch.Tensor:
+    """Differentiable L1 + SSIM loss (scalar); dL/dimage flows to image."""
+    return _L1Ssim.apply(image.contiguous(), target.contiguous(), lam, data_range)

@@ -1,0 +1,286 @@
+// L1 + SSIM training loss and its gradient dL/dI (the objective the reading
+// notes, section "Method", name as essential for PDR; constants of the usual
+// Gaussian-splatting form, see include/pdr.h):
+//
+//   L = (1 - lam) mean|I - T| + lam (1 - mean SSIM(I, T)),
+//   SSIM per (frame, channel) image with an 11 x 11 Gaussian window (sigma
+//   1.5), zero padding, C1 = (0.01 range)^2, C2 = (0.03 range)^2.
+//
+// k_loss_tile: one block per 32 x 32 output tile of one image.  The image and
+// the target are staged with a 10-pixel apron, shifted by a per-block
+// constant (the value at the tile centre): SSIM and its gradient are
+// invariant under that shift, and it keeps the fp32 variances and the final
+// gradient combination free of large cancellations.  Five separable window
+// sums (horizontal then vertical) give the moments mu_x, mu_y, E xx, E yy,
+// E xy on the tile plus a 5-pixel apron; there the SSIM map S and the
+// gradient coefficients
+//   A = dS/dmu_x - 2 mu_x dS/ds_xx - mu_y dS/ds_xy,  B = dS/ds_xx,  Cxy = dS/ds_xy
+// are formed (zero outside the image), and three more separable window sums
+// give dS_mean/dI = (G*A + 2 I (G*B) + T (G*Cxy)) / n on the tile.  Each block
+// leaves its partial sums of |I - T| and S in the workspace; k_loss_final
+// adds them in block order (fp64) into the loss.  Fixed order throughout:
+// bitwise reproducible.
+#include <math.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "pdr.h"
+
+namespace pdr {
+namespace {
+
+constexpr int kLT = 32;             // output tile edge
+constexpr int kLR = 5;              // window radius
+constexpr int kLW = 2 * kLR + 1;    // window taps
+constexpr int kLS = kLT + 2 * kLR;  // moment region edge (42)
+constexpr int kLI = kLT + 4 * kLR;  // staged input edge (52)
+constexpr int kLossThreads = 256;
+
+struct LossSmem {
+    float raw[kLW];               // Gaussian taps, sigma 1.5, before normalising
+    float taps[kLW];              // ... normalised to sum 1
+    float x[kLI][kLI];            // shifted image, zero-padded
+    float y[kLI][kLI];            // shifted target
+    float h[5][kLI][kLS];         // horizontal window sums (reused for the gradient pass)
+    float abc[3][kLS][kLS];       // A, B, Cxy on the tile and its apron
+    float red[2][kLossThreads / 32];
+};
+
+__global__ void __launch_bounds__(kLossThreads) k_loss_tile(
+    const float *__restrict__ img, const float *__restrict__ tgt, int BC, int H, int W, int TX,
+    int TY, float lam, float C1, float C2, double inv_n, float *__restrict__ grad,
+    float *__restrict__ part) {
+    extern __shared__ float4 lsm4[];
+    LossSmem &S = *reinterpret_cast<LossSmem *>(lsm4);
+    const int tid = threadIdx.x;
+    const int tiles = TX * TY;
+    const int im = blockIdx.x / tiles, t = blockIdx.x - im * tiles;
+    const int ty = t / TX, tx = t - ty * TX;
+    const int X0 = tx * kLT, Y0 = ty * kLT;
+    const size_t base = (size_t)im * H * W;
+    const float *ip = img + base, *tp = tgt + base;
+
+    if (tid < kLW) {
+        const float o = (float)(tid - kLR);
+        S.raw[tid] = expf(-(o * o) / (2.0f * 1.5f * 1.5f));
+    }
+    __syncthreads();
+    if (tid < kLW) {
+        float sum = 0.0f;
+        for (int d = 0; d < kLW; ++d) sum += S.raw[d];
+        S.taps[tid] = S.raw[tid] / sum;
+    }
+
+    // Shift: the values at the tile centre (clamped into the image).
+    const int cyy = min(Y0 + kLT / 2, H - 1), cxx = min(X0 + kLT / 2, W - 1);
+    const float sx = ip[(size_t)cyy * W + cxx], sy = tp[(size_t)cyy * W + cxx];
+
+    // 1. stage the shifted inputs over [Y0 - 10, Y0 + 41] x [X0 - 10, X0 + 41]
+    for (int i = tid; i < kLI * kLI; i += kLossThreads) {
+        const int r = i / kLI, c = i - r * kLI;
+        const int y = Y0 - 2 * kLR + r, x = X0 - 2 * kLR + c;
+        const bool in = y >= 0 && y < H && x >= 0 && x < W;
+        const size_t o = (size_t)y * W + x;
+        S.x[r][c] = (in ? ip[o] : 0.0f) - sx;
+        S.y[r][c] = (in ? tp[o] : 0.0f) - sy;
+    }
+    __syncthreads();
+
+    // 2. horizontal window sums of x, y, xx, yy, xy over all staged rows
+    for (int i = tid; i < kLI * kLS; i += kLossThreads) {
+        const int r = i / kLS, c = i - r * kLS;
+        float m0 = 0.f, m1 = 0.f, m2 = 0.f, m3 = 0.f, m4 = 0.f;
+#pragma unroll
+        for (int d = 0; d < kLW; ++d) {
+            const float g = S.taps[d], a = S.x[r][c + d], b = S.y[r][c + d];
+            const float ga = g * a, gb = g * b;
+            m0 += ga;
+            m1 += gb;
+            m2 = fmaf(ga, a, m2);
+            m3 = fmaf(gb, b, m3);
+            m4 = fmaf(ga, b, m4);
+        }
+        S.h[0][r][c] = m0;
+        S.h[1][r][c] = m1;
+        S.h[2][r][c] = m2;
+        S.h[3][r][c] = m3;
+        S.h[4][r][c] = m4;
+    }
+    __syncthreads();
+
+    // 3. vertical sums -> moments; SSIM map and gradient coefficients
+    float ssum = 0.0f;
+    for (int i = tid; i < kLS * kLS; i += kLossThreads) {
+        const int r = i / kLS, c = i - r * kLS;
+        const int y = Y0 - kLR + r, x = X0 - kLR + c;
+        float m[5] = {0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int d = 0; d < kLW; ++d) {
+            const float g = S.taps[d];
+#pragma unroll
+            for (int q = 0; q < 5; ++q) m[q] = fmaf(g, S.h[q][r + d][c], m[q]);
+        }
+        float A = 0.f, Bc = 0.f, Cc = 0.f;
+        if (y >= 0 && y < H && x >= 0 && x < W) {
+            const float mx = m[0], my = m[1];  // shifted means
+            const float vxx = fmaf(-mx, mx, m[2]), vyy = fmaf(-my, my, m[3]);
+            const float vxy = fmaf(-mx, my, m[4]);
+            const float ux = mx + sx, uy = my + sy;  // true means
+            const float N1 = fmaf(2.0f * ux, uy, C1), N2 = fmaf(2.0f, vxy, C2);
+            const float D1 = fmaf(ux, ux, fmaf(uy, uy, C1)), D2 = vxx + vyy + C2;
+            const float rD1 = 1.0f / D1, rD2 = 1.0f / D2, rD = rD1 * rD2;
+            const float s = N1 * N2 * rD;
+            const float dmu = 2.0f * uy * N2 * rD - 2.0f * ux * s * rD1;
+            Bc = -s * rD2;
+            Cc = 2.0f * N1 * rD;
+            A = dmu - 2.0f * mx * Bc - my * Cc;  // shifted means: the shift cancels exactly
+            if (r >= kLR && r < kLR + kLT && c >= kLR && c < kLR + kLT) ssum += s;
+        }
+        S.abc[0][r][c] = A;
+        S.abc[1][r][c] = Bc;
+        S.abc[2][r][c] = Cc;
+    }
+    __syncthreads();
+
+    // 4. horizontal window sums of A, B, Cxy over the moment rows
+    for (int i = tid; i < kLS * kLT; i += kLossThreads) {
+        const int r = i / kLT, c = i - r * kLT;
+        float a = 0.f, b = 0.f, e = 0.f;
+#pragma unroll
+        for (int d = 0; d < kLW; ++d) {
+            const float g = S.taps[d];
+            a = fmaf(g, S.abc[0][r][c + d], a);
+            b = fmaf(g, S.abc[1][r][c + d], b);
+            e = fmaf(g, S.abc[2][r][c + d], e);
+        }
+        S.h[0][r][c] = a;
+        S.h[1][r][c] = b;
+        S.h[2][r][c] = e;
+    }
+    __syncthreads();
+
+    // 5. vertical sums -> dL/dI on the tile
+    float lsum = 0.0f;
+    const float wl1 = (float)((1.0 - (double)lam) * inv_n), wss = (float)((double)lam * inv_n);
+    for (int i = tid; i < kLT * kLT; i += kLossThreads) {
+        const int r = i / kLT, c = i - r * kLT;
+        const int y = Y0 + r, x = X0 + c;
+        if (y >= H || x >= W) continue;
+        float a = 0.f, b = 0.f, e = 0.f;
+#pragma unroll
+        for (int d = 0; d < kLW; ++d) {
+            const float g = S.taps[d];
+            a = fmaf(g, S.h[0][r + d][c], a);
+            b = fmaf(g, S.h[1][r + d][c], b);
+            e = fmaf(g, S.h[2][r + d][c], e);
+        }
+        const float xs = S.x[r + 2 * kLR][c + 2 * kLR], ys = S.y[r + 2 * kLR][c + 2 * kLR];
+        const float dss = fmaf(2.0f * xs, b, fmaf(ys, e, a));  // n * dS_mean/dI
+        const size_t o = (size_t)y * W + x;
+        const float diff = ip[o] - tp[o];  // unshifted: ties stay exact zeros
+        const float sg = diff > 0.0f ? 1.0f : (diff < 0.0f ? -1.0f : 0.0f);
+        lsum += fabsf(diff);
+        grad[base + o] = fmaf(wl1, sg, -wss * dss);
+    }
+
+    // 6. block partial sums (fixed tree order)
+    const int lane = tid & 31, warp = tid >> 5;
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) {
+        lsum += __shfl_xor_sync(0xffffffffu, lsum, d);
+        ssum += __shfl_xor_sync(0xffffffffu, ssum, d);
+    }
+    if (lane == 0) {
+        S.red[0][warp] = lsum;
+        S.red[1][warp] = ssum;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        float l = 0.f, s = 0.f;
+        for (int w = 0; w < kLossThreads / 32; ++w) {
+            l += S.red[0][w];
+            s += S.red[1][w];
+        }
+        part[2 * (size_t)blockIdx.x] = l;
+        part[2 * (size_t)blockIdx.x + 1] = s;
+    }
+}
+
+// loss = (1 - lam) sum|I - T| / n + lam (1 - sum S / n), partials added in
+// block order in fp64 (each thread a contiguous range, then the threads in order).
+__global__ void __launch_bounds__(256) k_loss_final(const float *__restrict__ part, int nblocks,
+                                                    float lam, double inv_n,
+                                                    float *__restrict__ loss) {
+    __shared__ double sl[256], ss[256];
+    const int tid = threadIdx.x;
+    const int per = (nblocks + 255) / 256;
+    double l = 0.0, s = 0.0;
+    for (int j = tid * per; j < min(nblocks, (tid + 1) * per); ++j) {
+        l += part[2 * (size_t)j];
+        s += part[2 * (size_t)j + 1];
+    }
+    sl[tid] = l;
+    ss[tid] = s;
+    __syncthreads();
+    if (tid == 0) {
+        double L = 0.0, Sm = 0.0;
+        for (int j = 0; j < 256; ++j) {
+            L += sl[j];
+            Sm += ss[j];
+        }
+        *loss = (float)((1.0 - (double)lam) * L * inv_n + (double)lam * (1.0 - Sm * inv_n));
+    }
+}
+
+bool loss_geometry(int B, int C, int H, int W, int *TX, int *TY, long long *nblocks) {
+    if (B < 1 || C < 1 || H < 1 || W < 1) return false;
+    *TX = (W + kLT - 1) / kLT;
+    *TY = (H + kLT - 1) / kLT;
+    *nblocks = (long long)B * C * (*TX) * (*TY);
+    return *nblocks <= INT32_MAX && (long long)B * C * H * W <= (1ll << 40);
+}
+
+}  // namespace
+}  // namespace pdr
+
+using namespace pdr;
+
+extern "C" {
+
+size_t pdr_loss_workspace_bytes(int B, int C, int H, int W) {
+    int TX, TY;
+    long long nb;
+    if (!loss_geometry(B, C, H, W, &TX, &TY, &nb)) return 0;
+    return (size_t)(((2 * sizeof(float) * (size_t)nb) + 255) & ~(size_t)255);
+}
+
+pdr_status pdr_loss_l1_ssim(const float *image, const float *target, int B, int C, int H,
+                            int W, float lam, float data_range, float *loss, float *grad_image,
+                            void *workspace, size_t workspace_bytes, void *stream) {
+    int TX, TY;
+    long long nb;
+    if (!loss_geometry(B, C, H, W, &TX, &TY, &nb)) return PDR_ERR_INVALID_ARG;
+    if (!(lam >= 0.0f && lam <= 1.0f) || !(data_range > 0.0f) || !isfinite(data_range))
+        return PDR_ERR_INVALID_ARG;
+    if (!image || !target || !loss || !grad_image || !workspace) return PDR_ERR_INVALID_ARG;
+    if (((uintptr_t)image | (uintptr_t)target | (uintptr_t)loss | (uintptr_t)grad_image) & 3)
+        return PDR_ERR_INVALID_ARG;
+    if ((uintptr_t)workspace & 255) return PDR_ERR_INVALID_ARG;
+    if (workspace_bytes < pdr_loss_workspace_bytes(B, C, H, W)) return PDR_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t smem = sizeof(LossSmem);
+    if (cudaFuncSetAttribute(k_loss_tile, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+        return PDR_ERR_CUDA;
+    const double n = (double)B * C * H * W;
+    const float C1 = (0.01f * data_range) * (0.01f * data_range);
+    const float C2 = (0.03f * data_range) * (0.03f * data_range);
+    float *part = static_cast<float *>(workspace);
+    k_loss_tile<<<(unsigned)nb, kLossThreads, smem, s>>>(image, target, B * C, H, W, TX, TY, lam,
+                                                         C1, C2, 1.0 / n, grad_image, part);
+    if (cudaGetLastError() != cudaSuccess) return PDR_ERR_CUDA;
+    k_loss_final<<<1, 256, 0, s>>>(part, (int)nb, lam, 1.0 / n, loss);
+    return cudaGetLastError() == cudaSuccess ? PDR_OK : PDR_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -180,6 +180,38 @@ pdr_status pdr_render_fwd_noalloc(const float *params, int B, int N, int C, int 
  * clears it. */
 pdr_status pdr_check_device_error(void *workspace, void *stream);
 
+/* ---- Training loss: L1 + SSIM, producing dL/dI ------------------------------
+ * The objective the reading notes (section "Method", third point; "Key
+ * Insight / Why It Works") name as essential for PDR: an L1 term plus a
+ * structural-similarity term.  The pages give no weights or SSIM constants;
+ * the library takes the usual Gaussian-splatting ones:
+ *
+ *   L = (1 - lam) mean|I - T| + lam (1 - mean SSIM(I, T)),
+ *
+ * SSIM computed per (frame, channel) image with an 11 x 11 Gaussian window
+ * (sigma 1.5, taps normalised to sum 1), zero padding at the borders (maps of
+ * the image's size), C1 = (0.01 data_range)^2, C2 = (0.03 data_range)^2; the
+ * means run over all B*C*H*W elements.  dL/dI is the exact derivative of that
+ * definition (sign(0) = 0 for the L1 term); T gets no gradient. */
+
+/* Workspace bytes for pdr_loss_l1_ssim (per-block partial sums); 0 if the
+ * sizes are invalid. */
+size_t pdr_loss_workspace_bytes(int B, int C, int H, int W);
+
+/* image, target: [B][C][H][W] fp32 device; lam in [0, 1] (0.2 is the usual
+ * choice); data_range > 0 (1 for images in [0, 1]).  Writes the scalar loss to
+ * `loss` (one fp32 on the device) and dL/dimage to grad_image
+ * ([B][C][H][W], overwritten; it may not alias image or target).  The
+ * workspace (device, 256-byte aligned, pdr_loss_workspace_bytes) holds
+ * per-block partial sums, added in a fixed order: bitwise reproducible.
+ * Errors: PDR_ERR_INVALID_ARG for sizes < 1, lam outside [0, 1], a
+ * non-positive or non-finite data_range, null or misaligned pointers;
+ * PDR_ERR_WORKSPACE_TOO_SMALL; nothing is launched then.  Asynchronous on
+ * `stream` like the render calls. */
+pdr_status pdr_loss_l1_ssim(const float *image, const float *target, int B, int C, int H,
+                            int W, float lam, float data_range, float *loss, float *grad_image,
+                            void *workspace, size_t workspace_bytes, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

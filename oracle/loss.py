@@ -62,21 +62,22 @@ def window_2d(size: int = WINDOW, sigma: float = SIGMA) -> np.ndarray:
 
 def window_sum(img: np.ndarray, w2: np.ndarray) -> np.ndarray:
     """Zero-padded, same-size window sum out(p) = sum_o w2[o] img[p + o - r]
-    of one 2D image, written out over the window offsets (fp64)."""
+    over the last two axes of img (each 2D image on its own), written out
+    over the window offsets (fp64)."""
     kh, kw = w2.shape
     ry, rx = (kh - 1) // 2, (kw - 1) // 2
-    H, W = img.shape
-    pad = np.zeros((H + 2 * ry, W + 2 * rx), dtype=np.float64)
-    pad[ry:ry + H, rx:rx + W] = img
-    out = np.zeros((H, W), dtype=np.float64)
+    H, W = img.shape[-2:]
+    pad = np.zeros(img.shape[:-2] + (H + 2 * ry, W + 2 * rx), dtype=np.float64)
+    pad[..., ry:ry + H, rx:rx + W] = img
+    out = np.zeros(img.shape, dtype=np.float64)
     for dy in range(kh):
         for dx in range(kw):
-            out += w2[dy, dx] * pad[dy:dy + H, dx:dx + W]
+            out += w2[dy, dx] * pad[..., dy:dy + H, dx:dx + W]
     return out
 
 
 def ssim_parts(x: np.ndarray, y: np.ndarray, data_range: float = 1.0):
-    """Window moments and the SSIM map of one image pair (2D, fp64)."""
+    """Window moments and the SSIM map of image pairs (last two axes, fp64)."""
     w2 = window_2d()
     C1 = (K1 * data_range) ** 2
     C2 = (K2 * data_range) ** 2
@@ -108,20 +109,15 @@ def l1_ssim_loss(image: np.ndarray, target: np.ndarray, lam: float = DEFAULT_LAM
     w2 = window_2d()
     l1 = np.abs(x - y).sum() / n
     grad = (1.0 - lam) * np.sign(x - y) / n
-    ssim_total = 0.0
-    for b in range(B):
-        for c in range(C):
-            xi, yi = x[b, c], y[b, c]
-            P = ssim_parts(xi, yi, data_range)
-            S, N1, N2, D1, D2 = P["S"], P["N1"], P["N2"], P["D1"], P["D2"]
-            ssim_total += S.sum()
-            dS_dmx = 2.0 * P["my"] * N2 / (D1 * D2) - 2.0 * P["mx"] * S / D1
-            dS_dsxx = -S / D2
-            dS_dsxy = 2.0 * N1 / (D1 * D2)
-            A = dS_dmx - 2.0 * P["mx"] * dS_dsxx - P["my"] * dS_dsxy
-            dssim = (window_sum(A, w2) + 2.0 * xi * window_sum(dS_dsxx, w2)
-                     + yi * window_sum(dS_dsxy, w2)) / n
-            grad[b, c] -= lam * dssim
-    ssim_mean = ssim_total / n
+    P = ssim_parts(x, y, data_range)  # every (frame, channel) image on its own
+    S, N1, N2, D1, D2 = P["S"], P["N1"], P["N2"], P["D1"], P["D2"]
+    dS_dmx = 2.0 * P["my"] * N2 / (D1 * D2) - 2.0 * P["mx"] * S / D1
+    dS_dsxx = -S / D2
+    dS_dsxy = 2.0 * N1 / (D1 * D2)
+    A = dS_dmx - 2.0 * P["mx"] * dS_dsxx - P["my"] * dS_dsxy
+    dssim = (window_sum(A, w2) + 2.0 * x * window_sum(dS_dsxx, w2)
+             + y * window_sum(dS_dsxy, w2)) / n
+    grad -= lam * dssim
+    ssim_mean = S.sum() / n
     loss = (1.0 - lam) * l1 + lam * (1.0 - ssim_mean)
     return loss, grad, (l1, ssim_mean)

@@ -138,3 +138,26 @@ def test_python_api_surface():
                  "workspace_bytes", "check_device_error", "Workspace"]:
         assert callable(getattr(api, name)), name
     assert pkg.render is api.render
+
+
+def test_loss_workspace_sizes_and_validation_without_gpu():
+    """Loss entry points: sizes and argument checks that run before any launch."""
+    lib = _lib.load()
+    assert lib.pdr_loss_workspace_bytes(0, 1, 8, 8) == 0
+    assert lib.pdr_loss_workspace_bytes(1, 1, 8, -1) == 0
+    n1 = lib.pdr_loss_workspace_bytes(2, 3, 64, 96)      # 2 x 3 x 2 x 3 tiles, 2 floats each
+    assert n1 >= 2 * 4 * 36 and n1 % 256 == 0
+    assert lib.pdr_loss_workspace_bytes(2, 3, 65, 96) > n1 or lib.pdr_loss_workspace_bytes(2, 3, 65, 96) == n1
+    fake = 1 << 20  # never dereferenced: validation fails before any CUDA call
+    bad = [
+        (fake, fake, 0, 1, 8, 8, 0.2, 1.0, fake, fake, fake, 1 << 20, None),
+        (fake, fake, 1, 1, 8, 8, -0.1, 1.0, fake, fake, fake, 1 << 20, None),
+        (fake, fake, 1, 1, 8, 8, 0.2, float("nan"), fake, fake, fake, 1 << 20, None),
+        (0, fake, 1, 1, 8, 8, 0.2, 1.0, fake, fake, fake, 1 << 20, None),
+        (fake + 2, fake, 1, 1, 8, 8, 0.2, 1.0, fake, fake, fake, 1 << 20, None),
+        (fake, fake, 1, 1, 8, 8, 0.2, 1.0, fake, fake, fake + 16, 1 << 20, None),
+    ]
+    for args in bad:
+        assert lib.pdr_loss_l1_ssim(*args) == _lib.STATUS_CODES["PDR_ERR_INVALID_ARG"], args
+    assert lib.pdr_loss_l1_ssim(fake, fake, 1, 1, 8, 8, 0.2, 1.0, fake, fake, fake, 0, None) == \
+        _lib.STATUS_CODES["PDR_ERR_WORKSPACE_TOO_SMALL"]
