@@ -394,6 +394,80 @@ def time_e2e_steps(step, torch, K, stream):
     return np.array(out), h2d, d2h
 
 
+# FP32 instructions per pixel of the L1 + SSIM loss in its separable form:
+# x^2, y^2, xy (3); five moments, two 11-tap passes (110); SSIM map and the
+# three gradient coefficients (~25); three coefficient maps, two passes (66);
+# the final combination and the L1 term (6).
+LOSS_OPS_PER_PX = 210
+
+
+class LossBench:
+    """The L1 + SSIM loss on a workload's image shape: image ~ U[0, 1],
+    target = clip(image + N(0, 0.1)); one call per step, CUDA-graph replay,
+    CUDA events, L2 flushed before every call."""
+
+    def __init__(self, R, torch, w, seed, device):
+        rng = np.random.default_rng(seed + 7)
+        x = rng.uniform(0, 1, (w.B, w.C, w.H, w.W)).astype(np.float32)
+        y = np.clip(x + rng.normal(0, 0.1, x.shape), 0, 1).astype(np.float32)
+        self.x, self.y = x, y
+        self.xt, self.yt = torch.from_numpy(x).to(device), torch.from_numpy(y).to(device)
+        self.ws = torch.empty(max(R.loss_workspace_bytes(w.B, w.C, w.H, w.W), 256),
+                              dtype=torch.uint8, device=device)
+        self.grad = torch.empty_like(self.xt)
+        self.loss = torch.empty(1, dtype=torch.float32, device=device)
+        self.R, self.torch, self.px = R, torch, x.size
+        self.call()
+        torch.cuda.synchronize(device)
+        g = torch.cuda.CUDAGraph()
+        self.ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+        with torch.cuda.graph(g):
+            self.ev[0].record()
+            self.call()
+            self.ev[1].record()
+        self.graph = g
+
+    def call(self):
+        self.R.l1_ssim_loss(self.xt, self.yt, 0.2, 1.0, self.ws, self.grad, self.loss)
+
+    def time(self, flush, K, stream):
+        out = []
+        for _ in range(K):
+            flush.fill_(1)
+            self.graph.replay()
+            stream.synchronize()
+            out.append(self.ev[0].elapsed_time(self.ev[1]))
+        return float(np.mean(out))
+
+    def entry(self, ms, peak_tops):
+        ops = self.px * LOSS_OPS_PER_PX
+        achieved = ops / (ms * 1e-3) / 1e12
+        return {"ms_per_call": ms, "px_per_s": self.px / (ms * 1e-3),
+                "roofline": {"bound": "alu", "kernel": "k_loss_tile", "achieved": achieved,
+                             "peak": peak_tops, "unit": "Tinst/s", "frac": achieved / peak_tops,
+                             "ops_per_px": LOSS_OPS_PER_PX,
+                             "algorithmic_bytes": 12 * self.px},
+                "data": "image ~ U[0,1], target = clip(image + N(0, 0.1)), lam 0.2"}
+
+
+def loss_oracle_rate(x, y, seconds):
+    """fp64 oracle (numpy) pixels/s on whole frames of (x, y), about `seconds`."""
+    from oracle import loss as oracle_loss  # test infrastructure: the CPU-baseline leg only
+    reps, t0, px = 0, time.perf_counter(), 0
+    B = x.shape[0]
+    nf = 1
+    while True:
+        xs, ys = x[:nf], y[:nf]
+        oracle_loss.l1_ssim_loss(xs, ys)
+        reps += 1
+        px += xs.size
+        dt = time.perf_counter() - t0
+        if dt >= seconds:
+            break
+        nf = min(B, nf * 2)
+    return px / dt, "%d oracle calls on up to %d of %d frames (numpy fp64, 1 process)" % (reps, nf, B)
+
+
 def roofline_entry(kernel, ms, evals, C, peak_tops, workload, w):
     ops_f, ops_b = fp32_ops_per_eval(C)
     fwd = kernel.startswith("k_fwd")
@@ -494,6 +568,15 @@ def run_gpu(args, w):
                            % sm_max)
     other = roofline_entry(kern[1][1], kern[1][0], step.evals, w.C, peak_tops, w.name, w)
 
+    lb = LossBench(R, torch, w, rank_seed(w, rank), device)
+    loss_ms = lb.time(flush, args.steps, stream)
+    loss_entry = lb.entry(loss_ms, peak_tops)
+    if rank == 0 and world == 1 and args.cpu_seconds > 0:
+        rate, sample = loss_oracle_rate(lb.x, lb.y, min(3.0, args.cpu_seconds))
+        loss_entry["cpu_oracle_px_per_s"] = rate
+        loss_entry["cpu_oracle_sample"] = sample
+    del lb
+
     sweep = {}
     if args.sweep and rank == 0:
         for name in WORKLOAD_ORDER:
@@ -523,6 +606,11 @@ def run_gpu(args, w):
                 "step_frac": st.evals * (of + ob) / (tot * 1e-3) / 1e12 / peak_tops,
             }
             del st
+            lbs = LossBench(R, torch, sw, sw.seed, device)
+            lms = lbs.time(flush, args.sweep_steps, stream)
+            sweep[name]["ms_loss_l1_ssim"] = lms
+            sweep[name]["loss_frac"] = lbs.entry(lms, peak_tops)["roofline"]["frac"]
+            del lbs
 
     cpu = None
     if rank == 0 and world == 1 and args.cpu_seconds > 0:
@@ -557,6 +645,7 @@ def run_gpu(args, w):
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk,
             "cpu_baseline": cpu,
+            "loss_l1_ssim": loss_entry,
             "sweep": sweep,
         }
         print(json.dumps(line), flush=True)

@@ -222,7 +222,7 @@ def loss_workspace_bytes(B: int, C: int, H: int, W: int) -> int:
 
 def l1_ssim_loss(image: torch.Tensor, target: torch.Tensor, lam: float = 0.2,
                  data_range: float = 1.0, workspace: torch.Tensor | None = None,
-                 grad_out: torch.Tensor | None = None):
+                 grad_out: torch.Tensor | None = None, loss_out: torch.Tensor | None = None):
     """L1 + SSIM training loss and dL/dimage (see pdr_loss_l1_ssim).
 
     image, target: contiguous fp32 CUDA tensors [B, C, H, W].  Returns
@@ -241,7 +241,7 @@ def l1_ssim_loss(image: torch.Tensor, target: torch.Tensor, lam: float = 0.2,
     if workspace is None or workspace.numel() < nb:
         workspace = torch.empty(max(nb, 256), dtype=torch.uint8, device=dev)
     grad = torch.empty_like(image) if grad_out is None else grad_out
-    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    loss = torch.empty(1, dtype=torch.float32, device=dev) if loss_out is None else loss_out
     _lib.check("pdr_loss_l1_ssim", lib.pdr_loss_l1_ssim(
         _ptr(image), _ptr(target), B, C, H, W, float(lam), float(data_range), _ptr(loss),
         _ptr(grad), _ptr(workspace), workspace.numel(), _stream(dev)))

@@ -34,7 +34,8 @@ constexpr int kLR = 5;              // window radius
 constexpr int kLW = 2 * kLR + 1;    // window taps
 constexpr int kLS = kLT + 2 * kLR;  // moment region edge (42)
 constexpr int kLI = kLT + 4 * kLR;  // staged input edge (52)
-constexpr int kLossThreads = 256;
+constexpr int kLossThreads = 512;
+constexpr int kLU = (kLI * kLI + kLossThreads - 1) / kLossThreads;  // staged pixels per thread
 
 struct LossSmem {
     float raw[kLW];               // Gaussian taps, sigma 1.5, before normalising
@@ -43,6 +44,7 @@ struct LossSmem {
     float y[kLI][kLI];            // shifted target
     float h[5][kLI][kLS];         // horizontal window sums (reused for the gradient pass)
     float abc[3][kLS][kLS];       // A, B, Cxy on the tile and its apron
+    signed char sgn[kLT][kLT];    // sign(I - T) on the tile
     float red[2][kLossThreads / 32];
 };
 
@@ -76,13 +78,35 @@ __global__ void __launch_bounds__(kLossThreads) k_loss_tile(
     const float sx = ip[(size_t)cyy * W + cxx], sy = tp[(size_t)cyy * W + cxx];
 
     // 1. stage the shifted inputs over [Y0 - 10, Y0 + 41] x [X0 - 10, X0 + 41]
-    for (int i = tid; i < kLI * kLI; i += kLossThreads) {
-        const int r = i / kLI, c = i - r * kLI;
-        const int y = Y0 - 2 * kLR + r, x = X0 - 2 * kLR + c;
-        const bool in = y >= 0 && y < H && x >= 0 && x < W;
-        const size_t o = (size_t)y * W + x;
-        S.x[r][c] = (in ? ip[o] : 0.0f) - sx;
-        S.y[r][c] = (in ? tp[o] : 0.0f) - sy;
+    //    (all of a thread's loads in flight together); the L1 term of the
+    //    tile's own pixels is taken from the unshifted values here.
+    float lsum = 0.0f;
+    {
+        float xv[kLU], yv[kLU];
+#pragma unroll
+        for (int u = 0; u < kLU; ++u) {
+            const int i = u * kLossThreads + tid;
+            const int r = i / kLI, c = i - r * kLI;
+            const int y = Y0 - 2 * kLR + r, x = X0 - 2 * kLR + c;
+            const bool in = i < kLI * kLI && y >= 0 && y < H && x >= 0 && x < W;
+            const size_t o = in ? (size_t)y * W + x : 0;
+            xv[u] = in ? ip[o] : 0.0f;
+            yv[u] = in ? tp[o] : 0.0f;
+        }
+#pragma unroll
+        for (int u = 0; u < kLU; ++u) {
+            const int i = u * kLossThreads + tid;
+            if (i >= kLI * kLI) continue;
+            const int r = i / kLI, c = i - r * kLI;
+            S.x[r][c] = xv[u] - sx;
+            S.y[r][c] = yv[u] - sy;
+            const int tr = r - 2 * kLR, tc = c - 2 * kLR;
+            if (tr >= 0 && tr < kLT && tc >= 0 && tc < kLT) {
+                const float diff = xv[u] - yv[u];  // unshifted: ties stay exact zeros
+                S.sgn[tr][tc] = diff > 0.0f ? 1 : (diff < 0.0f ? -1 : 0);
+                if (Y0 + tr < H && X0 + tc < W) lsum += fabsf(diff);
+            }
+        }
     }
     __syncthreads();
 
@@ -160,7 +184,6 @@ __global__ void __launch_bounds__(kLossThreads) k_loss_tile(
     __syncthreads();
 
     // 5. vertical sums -> dL/dI on the tile
-    float lsum = 0.0f;
     const float wl1 = (float)((1.0 - (double)lam) * inv_n), wss = (float)((double)lam * inv_n);
     for (int i = tid; i < kLT * kLT; i += kLossThreads) {
         const int r = i / kLT, c = i - r * kLT;
@@ -176,11 +199,7 @@ __global__ void __launch_bounds__(kLossThreads) k_loss_tile(
         }
         const float xs = S.x[r + 2 * kLR][c + 2 * kLR], ys = S.y[r + 2 * kLR][c + 2 * kLR];
         const float dss = fmaf(2.0f * xs, b, fmaf(ys, e, a));  // n * dS_mean/dI
-        const size_t o = (size_t)y * W + x;
-        const float diff = ip[o] - tp[o];  // unshifted: ties stay exact zeros
-        const float sg = diff > 0.0f ? 1.0f : (diff < 0.0f ? -1.0f : 0.0f);
-        lsum += fabsf(diff);
-        grad[base + o] = fmaf(wl1, sg, -wss * dss);
+        grad[base + (size_t)y * W + x] = fmaf(wl1, (float)S.sgn[r][c], -wss * dss);
     }
 
     // 6. block partial sums (fixed tree order)
