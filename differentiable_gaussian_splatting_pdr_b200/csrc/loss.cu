@@ -38,8 +38,6 @@ constexpr int kLossThreads = 512;
 constexpr int kLU = (kLI * kLI + kLossThreads - 1) / kLossThreads;  // staged pixels per thread
 
 struct LossSmem {
-    float raw[kLW];               // Gaussian taps, sigma 1.5, before normalising
-    float taps[kLW];              // ... normalised to sum 1
     float x[kLI][kLI];            // shifted image, zero-padded
     float y[kLI][kLI];            // shifted target
     float h[5][kLI][kLS];         // horizontal window sums (reused for the gradient pass)
@@ -48,10 +46,23 @@ struct LossSmem {
     float red[2][kLossThreads / 32];
 };
 
+// The window taps travel as a kernel argument (constant bank): every FMA
+// reads its tap without a shared-memory load.
+struct Taps {
+    float t[kLW];
+};
+
+// Register-blocked passes: a thread produces RB neighbouring outputs of a
+// window sum from one streamed read of the RB + 10 inputs they share.
+constexpr int kRB2 = 6;  // horizontal moments: 42 = 7 x 6 outputs per row
+constexpr int kRB3 = 3;  // vertical moments:   42 = 14 x 3 outputs per column
+constexpr int kRB4 = 4;  // horizontal coefficients: 32 = 8 x 4
+constexpr int kRB5 = 2;  // vertical coefficients:   32 = 16 x 2
+
 __global__ void __launch_bounds__(kLossThreads) k_loss_tile(
     const float *__restrict__ img, const float *__restrict__ tgt, int BC, int H, int W, int TX,
-    int TY, float lam, float C1, float C2, double inv_n, float *__restrict__ grad,
-    float *__restrict__ part) {
+    int TY, float lam, float C1, float C2, double inv_n, const Taps tp_,
+    float *__restrict__ grad, float *__restrict__ part) {
     extern __shared__ float4 lsm4[];
     LossSmem &S = *reinterpret_cast<LossSmem *>(lsm4);
     const int tid = threadIdx.x;
@@ -61,17 +72,7 @@ __global__ void __launch_bounds__(kLossThreads) k_loss_tile(
     const int X0 = tx * kLT, Y0 = ty * kLT;
     const size_t base = (size_t)im * H * W;
     const float *ip = img + base, *tp = tgt + base;
-
-    if (tid < kLW) {
-        const float o = (float)(tid - kLR);
-        S.raw[tid] = expf(-(o * o) / (2.0f * 1.5f * 1.5f));
-    }
-    __syncthreads();
-    if (tid < kLW) {
-        float sum = 0.0f;
-        for (int d = 0; d < kLW; ++d) sum += S.raw[d];
-        S.taps[tid] = S.raw[tid] / sum;
-    }
+    const float *g = tp_.t;
 
     // Shift: the values at the tile centre (clamped into the image).
     const int cyy = min(Y0 + kLT / 2, H - 1), cxx = min(X0 + kLT / 2, W - 1);
@@ -111,95 +112,143 @@ __global__ void __launch_bounds__(kLossThreads) k_loss_tile(
     __syncthreads();
 
     // 2. horizontal window sums of x, y, xx, yy, xy over all staged rows
-    for (int i = tid; i < kLI * kLS; i += kLossThreads) {
-        const int r = i / kLS, c = i - r * kLS;
-        float m0 = 0.f, m1 = 0.f, m2 = 0.f, m3 = 0.f, m4 = 0.f;
+    for (int it = tid; it < kLI * (kLS / kRB2); it += kLossThreads) {
+        const int r = it / (kLS / kRB2), c0 = (it - r * (kLS / kRB2)) * kRB2;
+        float m[5][kRB2];
 #pragma unroll
-        for (int d = 0; d < kLW; ++d) {
-            const float g = S.taps[d], a = S.x[r][c + d], b = S.y[r][c + d];
-            const float ga = g * a, gb = g * b;
-            m0 += ga;
-            m1 += gb;
-            m2 = fmaf(ga, a, m2);
-            m3 = fmaf(gb, b, m3);
-            m4 = fmaf(ga, b, m4);
+        for (int j = 0; j < kRB2; ++j)
+#pragma unroll
+            for (int q = 0; q < 5; ++q) m[q][j] = 0.0f;
+#pragma unroll
+        for (int k = 0; k < kRB2 + kLW - 1; ++k) {
+            const float a = S.x[r][c0 + k], b = S.y[r][c0 + k];
+            const float aa = a * a, bb = b * b, ab = a * b;
+#pragma unroll
+            for (int j = 0; j < kRB2; ++j) {
+                const int d = k - j;  // tap of output c0 + j
+                if (d < 0 || d >= kLW) continue;
+                m[0][j] = fmaf(g[d], a, m[0][j]);
+                m[1][j] = fmaf(g[d], b, m[1][j]);
+                m[2][j] = fmaf(g[d], aa, m[2][j]);
+                m[3][j] = fmaf(g[d], bb, m[3][j]);
+                m[4][j] = fmaf(g[d], ab, m[4][j]);
+            }
         }
-        S.h[0][r][c] = m0;
-        S.h[1][r][c] = m1;
-        S.h[2][r][c] = m2;
-        S.h[3][r][c] = m3;
-        S.h[4][r][c] = m4;
+#pragma unroll
+        for (int q = 0; q < 5; ++q)
+#pragma unroll
+            for (int j = 0; j < kRB2; ++j) S.h[q][r][c0 + j] = m[q][j];
     }
     __syncthreads();
 
     // 3. vertical sums -> moments; SSIM map and gradient coefficients
     float ssum = 0.0f;
-    for (int i = tid; i < kLS * kLS; i += kLossThreads) {
-        const int r = i / kLS, c = i - r * kLS;
-        const int y = Y0 - kLR + r, x = X0 - kLR + c;
-        float m[5] = {0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int it = tid; it < (kLS / kRB3) * kLS; it += kLossThreads) {
+        const int rb = it / kLS, c = it - rb * kLS, r0 = rb * kRB3;
+        float m[5][kRB3];
 #pragma unroll
-        for (int d = 0; d < kLW; ++d) {
-            const float g = S.taps[d];
+        for (int j = 0; j < kRB3; ++j)
 #pragma unroll
-            for (int q = 0; q < 5; ++q) m[q] = fmaf(g, S.h[q][r + d][c], m[q]);
+            for (int q = 0; q < 5; ++q) m[q][j] = 0.0f;
+#pragma unroll
+        for (int k = 0; k < kRB3 + kLW - 1; ++k) {
+            float v[5];
+#pragma unroll
+            for (int q = 0; q < 5; ++q) v[q] = S.h[q][r0 + k][c];
+#pragma unroll
+            for (int j = 0; j < kRB3; ++j) {
+                const int d = k - j;
+                if (d < 0 || d >= kLW) continue;
+#pragma unroll
+                for (int q = 0; q < 5; ++q) m[q][j] = fmaf(g[d], v[q], m[q][j]);
+            }
         }
-        float A = 0.f, Bc = 0.f, Cc = 0.f;
-        if (y >= 0 && y < H && x >= 0 && x < W) {
-            const float mx = m[0], my = m[1];  // shifted means
-            const float vxx = fmaf(-mx, mx, m[2]), vyy = fmaf(-my, my, m[3]);
-            const float vxy = fmaf(-mx, my, m[4]);
-            const float ux = mx + sx, uy = my + sy;  // true means
-            const float N1 = fmaf(2.0f * ux, uy, C1), N2 = fmaf(2.0f, vxy, C2);
-            const float D1 = fmaf(ux, ux, fmaf(uy, uy, C1)), D2 = vxx + vyy + C2;
-            const float rD1 = 1.0f / D1, rD2 = 1.0f / D2, rD = rD1 * rD2;
-            const float s = N1 * N2 * rD;
-            const float dmu = 2.0f * uy * N2 * rD - 2.0f * ux * s * rD1;
-            Bc = -s * rD2;
-            Cc = 2.0f * N1 * rD;
-            A = dmu - 2.0f * mx * Bc - my * Cc;  // shifted means: the shift cancels exactly
-            if (r >= kLR && r < kLR + kLT && c >= kLR && c < kLR + kLT) ssum += s;
+#pragma unroll
+        for (int j = 0; j < kRB3; ++j) {
+            const int r = r0 + j;
+            const int y = Y0 - kLR + r, x = X0 - kLR + c;
+            float A = 0.f, Bc = 0.f, Cc = 0.f;
+            if (y >= 0 && y < H && x >= 0 && x < W) {
+                const float mx = m[0][j], my = m[1][j];  // shifted means
+                const float vxx = fmaf(-mx, mx, m[2][j]), vyy = fmaf(-my, my, m[3][j]);
+                const float vxy = fmaf(-mx, my, m[4][j]);
+                const float ux = mx + sx, uy = my + sy;  // true means
+                const float N1 = fmaf(2.0f * ux, uy, C1), N2 = fmaf(2.0f, vxy, C2);
+                const float D1 = fmaf(ux, ux, fmaf(uy, uy, C1)), D2 = vxx + vyy + C2;
+                const float rD1 = 1.0f / D1, rD2 = 1.0f / D2, rD = rD1 * rD2;
+                const float s = N1 * N2 * rD;
+                const float dmu = 2.0f * uy * N2 * rD - 2.0f * ux * s * rD1;
+                Bc = -s * rD2;
+                Cc = 2.0f * N1 * rD;
+                A = dmu - 2.0f * mx * Bc - my * Cc;  // shifted means: the shift cancels exactly
+                if (r >= kLR && r < kLR + kLT && c >= kLR && c < kLR + kLT) ssum += s;
+            }
+            S.abc[0][r][c] = A;
+            S.abc[1][r][c] = Bc;
+            S.abc[2][r][c] = Cc;
         }
-        S.abc[0][r][c] = A;
-        S.abc[1][r][c] = Bc;
-        S.abc[2][r][c] = Cc;
     }
     __syncthreads();
 
     // 4. horizontal window sums of A, B, Cxy over the moment rows
-    for (int i = tid; i < kLS * kLT; i += kLossThreads) {
-        const int r = i / kLT, c = i - r * kLT;
-        float a = 0.f, b = 0.f, e = 0.f;
+    for (int it = tid; it < kLS * (kLT / kRB4); it += kLossThreads) {
+        const int r = it / (kLT / kRB4), c0 = (it - r * (kLT / kRB4)) * kRB4;
+        float m[3][kRB4];
 #pragma unroll
-        for (int d = 0; d < kLW; ++d) {
-            const float g = S.taps[d];
-            a = fmaf(g, S.abc[0][r][c + d], a);
-            b = fmaf(g, S.abc[1][r][c + d], b);
-            e = fmaf(g, S.abc[2][r][c + d], e);
+        for (int j = 0; j < kRB4; ++j)
+#pragma unroll
+            for (int q = 0; q < 3; ++q) m[q][j] = 0.0f;
+#pragma unroll
+        for (int k = 0; k < kRB4 + kLW - 1; ++k) {
+            float v[3];
+#pragma unroll
+            for (int q = 0; q < 3; ++q) v[q] = S.abc[q][r][c0 + k];
+#pragma unroll
+            for (int j = 0; j < kRB4; ++j) {
+                const int d = k - j;
+                if (d < 0 || d >= kLW) continue;
+#pragma unroll
+                for (int q = 0; q < 3; ++q) m[q][j] = fmaf(g[d], v[q], m[q][j]);
+            }
         }
-        S.h[0][r][c] = a;
-        S.h[1][r][c] = b;
-        S.h[2][r][c] = e;
+#pragma unroll
+        for (int q = 0; q < 3; ++q)
+#pragma unroll
+            for (int j = 0; j < kRB4; ++j) S.h[q][r][c0 + j] = m[q][j];
     }
     __syncthreads();
 
     // 5. vertical sums -> dL/dI on the tile
     const float wl1 = (float)((1.0 - (double)lam) * inv_n), wss = (float)((double)lam * inv_n);
-    for (int i = tid; i < kLT * kLT; i += kLossThreads) {
-        const int r = i / kLT, c = i - r * kLT;
-        const int y = Y0 + r, x = X0 + c;
-        if (y >= H || x >= W) continue;
-        float a = 0.f, b = 0.f, e = 0.f;
+    for (int it = tid; it < (kLT / kRB5) * kLT; it += kLossThreads) {
+        const int rb = it / kLT, c = it - rb * kLT, r0 = rb * kRB5;
+        float m[3][kRB5];
 #pragma unroll
-        for (int d = 0; d < kLW; ++d) {
-            const float g = S.taps[d];
-            a = fmaf(g, S.h[0][r + d][c], a);
-            b = fmaf(g, S.h[1][r + d][c], b);
-            e = fmaf(g, S.h[2][r + d][c], e);
+        for (int j = 0; j < kRB5; ++j)
+#pragma unroll
+            for (int q = 0; q < 3; ++q) m[q][j] = 0.0f;
+#pragma unroll
+        for (int k = 0; k < kRB5 + kLW - 1; ++k) {
+            float v[3];
+#pragma unroll
+            for (int q = 0; q < 3; ++q) v[q] = S.h[q][r0 + k][c];
+#pragma unroll
+            for (int j = 0; j < kRB5; ++j) {
+                const int d = k - j;
+                if (d < 0 || d >= kLW) continue;
+#pragma unroll
+                for (int q = 0; q < 3; ++q) m[q][j] = fmaf(g[d], v[q], m[q][j]);
+            }
         }
-        const float xs = S.x[r + 2 * kLR][c + 2 * kLR], ys = S.y[r + 2 * kLR][c + 2 * kLR];
-        const float dss = fmaf(2.0f * xs, b, fmaf(ys, e, a));  // n * dS_mean/dI
-        grad[base + (size_t)y * W + x] = fmaf(wl1, (float)S.sgn[r][c], -wss * dss);
+#pragma unroll
+        for (int j = 0; j < kRB5; ++j) {
+            const int r = r0 + j;
+            const int y = Y0 + r, x = X0 + c;
+            if (y >= H || x >= W) continue;
+            const float xs = S.x[r + 2 * kLR][c + 2 * kLR], ys = S.y[r + 2 * kLR][c + 2 * kLR];
+            const float dss = fmaf(2.0f * xs, m[1][j], fmaf(ys, m[2][j], m[0][j]));  // n * dS_mean/dI
+            grad[base + (size_t)y * W + x] = fmaf(wl1, (float)S.sgn[r][c], -wss * dss);
+        }
     }
 
     // 6. block partial sums (fixed tree order)
@@ -295,8 +344,19 @@ pdr_status pdr_loss_l1_ssim(const float *image, const float *target, int B, int 
     const float C1 = (0.01f * data_range) * (0.01f * data_range);
     const float C2 = (0.03f * data_range) * (0.03f * data_range);
     float *part = static_cast<float *>(workspace);
+    // Window taps exp(-d^2 / (2 sigma^2)), sigma 1.5, normalised to sum 1.
+    Taps taps;
+    {
+        double v[kLW], sum = 0.0;
+        for (int d = 0; d < kLW; ++d) {
+            const double o = d - kLR;
+            v[d] = exp(-(o * o) / (2.0 * 1.5 * 1.5));
+            sum += v[d];
+        }
+        for (int d = 0; d < kLW; ++d) taps.t[d] = (float)(v[d] / sum);
+    }
     k_loss_tile<<<(unsigned)nb, kLossThreads, smem, s>>>(image, target, B * C, H, W, TX, TY, lam,
-                                                         C1, C2, 1.0 / n, grad_image, part);
+                                                         C1, C2, 1.0 / n, taps, grad_image, part);
     if (cudaGetLastError() != cudaSuccess) return PDR_ERR_CUDA;
     k_loss_final<<<1, 256, 0, s>>>(part, (int)nb, lam, 1.0 / n, loss);
     return cudaGetLastError() == cudaSuccess ? PDR_OK : PDR_ERR_CUDA;
