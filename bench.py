@@ -612,6 +612,24 @@ def run_gpu(args, w):
             sweep[name]["loss_frac"] = lbs.entry(lms, peak_tops)["roofline"]["frac"]
             del lbs
 
+    knobs = {}
+    if args.knobs and args.sweep and rank == 0:
+        from differentiable_gaussian_splatting_pdr_b200.inputs import knob_workloads
+        for name, kw in knob_workloads(w.name if w.name in ("mono64",) else "mono64").items():
+            st = Step(R, torch, kw, kw.seed, device)
+            st.capture()
+            for _ in range(5):
+                flush.fill_(1)
+                st.replay()
+            pr = time_graph(st, "main", flush, args.sweep_steps, stream)
+            R.check_device_error(st.ws, device)
+            tot = float(pr[:, 0].mean())
+            of, ob = fp32_ops_per_eval(kw.C)
+            knobs[name] = {"desc": kw.desc, "evals_per_step": st.evals, "ms_per_step": tot,
+                           "evals_per_s": st.evals / (tot * 1e-3),
+                           "step_frac": st.evals * (of + ob) / (tot * 1e-3) / 1e12 / peak_tops}
+            del st
+
     cpu = None
     if rank == 0 and world == 1 and args.cpu_seconds > 0:
         v, fps, cores, sample, _ = oracle_sample(w, args.cpu_seconds)
@@ -647,6 +665,7 @@ def run_gpu(args, w):
             "cpu_baseline": cpu,
             "loss_l1_ssim": loss_entry,
             "sweep": sweep,
+            "knobs": knobs,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -668,6 +687,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="host-core time budget of the oracle baseline (0 = skip)")
     ap.add_argument("--no-sweep", dest="sweep", action="store_false")
+    ap.add_argument("--no-knobs", dest="knobs", action="store_false",
+                    help="skip the knob variants (grid layout, Gaussian count, window size)")
     ap.add_argument("--sweep-steps", type=int, default=50)
     args = ap.parse_args()
     if args.warmup < 3:

@@ -15,7 +15,8 @@ which are not available here: only their shapes (frames, channels, grid,
 Gaussians per frame, window size) are mimicked.
 
 Draw order per workload (numpy PCG64 ``default_rng(seed)``, fp64 draws cast
-to fp32 once): mu_x ~ U[0, W), mu_y ~ U[0, H), s_1, s_2 ~ N(m, sd),
+to fp32 once): mu_x ~ U[0, W), mu_y ~ U[0, H) (or, for the grid layout, the
+jitters of a regular grid), s_1, s_2 ~ N(m, sd),
 theta ~ U[0, pi), a (row-major [B, N, C]), then dL/dI ~ N(0, 1) as [B, C, H, W].
 """
 from __future__ import annotations
@@ -40,6 +41,7 @@ class Workload:
     amp: Tuple[str, float, float] = ("normal", 0.0, 1.0)  # (kind, p0, p1)
     seed: int = 0
     desc: str = ""
+    layout: str = "uniform"  # "uniform" means, or "grid": a jittered regular grid
 
     @property
     def P(self) -> int:
@@ -81,11 +83,31 @@ WORKLOADS: Dict[str, Workload] = {
 WORKLOAD_ORDER = ["tiny", "mono64", "rgb128", "field32x64", "stress512"]
 
 
+def _grid_means(rng, w: Workload):
+    """Grid-initialised means (the initial layout of a Gaussian field): the N
+    Gaussians of a frame on the first N cells of a ceil(sqrt(N W / H)) x
+    ceil(N / that) grid over the frame, each jittered U(-1/4, 1/4) of a cell."""
+    B, N = w.B, w.N
+    gx = max(1, int(np.ceil(np.sqrt(N * w.W / w.H))))
+    gy = max(1, int(np.ceil(N / gx)))
+    cell = np.arange(N)
+    cx = (cell % gx + 0.5) * (w.W / gx)
+    cy = (cell // gx + 0.5) * (w.H / gy)
+    jx = rng.uniform(-0.25, 0.25, size=(B, N)) * (w.W / gx)
+    jy = rng.uniform(-0.25, 0.25, size=(B, N)) * (w.H / gy)
+    return cx[None, :] + jx, cy[None, :] + jy
+
+
 def _draw(w: Workload, seed, want_grad: bool):
     rng = np.random.default_rng(w.seed if seed is None else seed)
     B, N, C = w.B, w.N, w.C
-    mu_x = rng.uniform(0.0, float(w.W), size=(B, N))
-    mu_y = rng.uniform(0.0, float(w.H), size=(B, N))
+    if w.layout == "grid":
+        mu_x, mu_y = _grid_means(rng, w)
+    elif w.layout == "uniform":
+        mu_x = rng.uniform(0.0, float(w.W), size=(B, N))
+        mu_y = rng.uniform(0.0, float(w.H), size=(B, N))
+    else:
+        raise ValueError(w.layout)
     s1 = rng.normal(w.s_mean, w.s_std, size=(B, N))
     s2 = rng.normal(w.s_mean, w.s_std, size=(B, N))
     theta = rng.uniform(0.0, np.pi, size=(B, N))
@@ -122,6 +144,22 @@ def make_grad_image(w: Workload, seed: int | None = None) -> np.ndarray:
 def make_inputs(w: Workload, seed: int | None = None):
     """(params [B,N,5+C], grad_image [B,C,H,W]) for a workload, fp32."""
     return _draw(w, seed, True)
+
+
+def knob_workloads(base: str = "mono64"):
+    """Variants of one workload along the knobs the pages name (reading notes,
+    "Relation To Prior Work" and "Limitation": grid-initialised Gaussians, the
+    Gaussian count and the kernel support): name -> Workload."""
+    w = WORKLOADS[base]
+    out = {"%s-grid" % base: replace(w, layout="grid", name="%s-grid" % base,
+                                      desc=w.desc + ", grid-initialised means")}
+    for n in (w.N // 4, w.N * 4):
+        out["%s-N%d" % (base, n)] = replace(w, N=n, name="%s-N%d" % (base, n),
+                                              desc="%s with N=%d" % (w.desc, n))
+    for k in (5, 13, 17):
+        out["%s-k%d" % (base, k)] = replace(w, k=k, name="%s-k%d" % (base, k),
+                                              desc="%s with k=%d" % (w.desc, k))
+    return out
 
 
 def rank_seed(w: Workload, rank: int) -> int:

@@ -241,3 +241,13 @@ def test_many_small_frames(B):
     w = WORKLOADS["field32x64"].scaled(B=B, N=300)
     p, g = make_inputs(w)
     check_all(p, g, w.H, w.W, w.k)
+
+
+@pytest.mark.parametrize("name", ["mono64-grid", "mono64-N256", "mono64-N4096", "mono64-k5",
+                                  "mono64-k13", "mono64-k17"])
+def test_knob_workloads(name):
+    """The knobs the pages name: grid-initialised means, Gaussian count, window size."""
+    from differentiable_gaussian_splatting_pdr_b200.inputs import knob_workloads
+    w = knob_workloads()[name]
+    p, g = make_inputs(w)
+    check_all(p, g, w.H, w.W, w.k)

@@ -371,3 +371,20 @@ def test_binning_matches_window_indicators(H, W, k, seed):
     got = [ids[offs[t]:offs[t + 1]].tolist() for t in range(TX * TY)]
     assert got == want
     assert offs[-1] == len(ids) == sum(len(x) for x in want)
+
+
+def test_grid_layout_puts_one_gaussian_per_cell():
+    """Knob workloads: the grid-initialised layout is seeded, inside the frame,
+    and holds exactly one mean per grid cell (jitter under half a cell)."""
+    from differentiable_gaussian_splatting_pdr_b200.inputs import knob_workloads, make_inputs
+    w = knob_workloads()["mono64-grid"]
+    p1, _ = make_inputs(w)
+    p2, _ = make_inputs(w)
+    assert np.array_equal(p1, p2)
+    mx, my = p1[..., 0].astype(np.float64), p1[..., 1].astype(np.float64)
+    assert mx.min() >= 0 and mx.max() < w.W and my.min() >= 0 and my.max() < w.H
+    gx = int(np.ceil(np.sqrt(w.N * w.W / w.H)))
+    gy = int(np.ceil(w.N / gx))
+    cell = np.floor(my / (w.H / gy)) * gx + np.floor(mx / (w.W / gx))
+    for b in range(w.B):
+        assert np.array_equal(np.sort(cell[b]), np.arange(w.N))
