@@ -36,7 +36,8 @@ namespace pdr {
 
 namespace {
 
-constexpr int kFwdBatch = 64;          // entries staged per batch (byte offsets fit 16 bits)
+constexpr int kFwdBatch = 64;          // entries staged per batch by k_fwd (byte offsets fit 16 bits)
+constexpr int kClusterBatch = 128;     // ... and by k_fwd_cluster (fewer batch barriers)
 constexpr int kClusterListCap = 1024;  // tile-list entries a clustered block keeps on chip
 constexpr int kChunkSmem = 256;        // Gaussians per clustered block whose records stay on chip
 
@@ -53,11 +54,11 @@ struct FwdLayout {
 };
 
 // Shared-memory buffers of one rendering block.
-template <int C>
+template <int C, int NB>
 struct FwdSmem {
-    float4 rec[kFwdBatch * FwdRec<C>::kVec];
-    unsigned win[kFwdBatch];  // window as column bits | row bits << 16 (tile pixels)
-    unsigned sub[16][kFwdBatch];
+    float4 rec[NB * FwdRec<C>::kVec];
+    unsigned win[NB];  // window as column bits | row bits << 16 (tile pixels)
+    unsigned sub[16][NB];
     int subn[16];
 };
 
@@ -65,10 +66,10 @@ struct FwdSmem {
 // (X0, Y0) of frame b into acc.  Called by the whole block.
 // fetch(i, A, Q, amp) supplies the record and amplitudes of frame-local
 // Gaussian i (from global memory, or from a cluster peer's shared memory).
-template <int C, int PL, typename Fetch>
+template <int C, int PL, int NB, typename Fetch>
 __device__ __forceinline__ void render_list(const Geom &g, Fetch fetch, const int *list,
                                             int L, int X0, int Y0, int *err,
-                                            FwdSmem<C> &S, float (&acc)[PL][C]) {
+                                            FwdSmem<C, NB> &S, float (&acc)[PL][C]) {
     using LY = FwdLayout<PL>;
     constexpr int RV = FwdRec<C>::kVec;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -79,8 +80,9 @@ __device__ __forceinline__ void render_list(const Geom &g, Fetch fetch, const in
     const int bitshift = 16 + 4 * lrow + lcol;  // this lane's bits of a packed sub-list entry
 
     const unsigned lt = lanemask_lt();
-    for (int e0 = 0; e0 < L; e0 += kFwdBatch) {
-        const int n = min(kFwdBatch, L - e0);
+    static_assert(NB * FwdRec<C>::kVec * 16 <= 65536, "record offsets must fit 16 bits");
+    for (int e0 = 0; e0 < L; e0 += NB) {
+        const int n = min(NB, L - e0);
         __syncthreads();  // the previous batch is fully consumed
         for (int e = tid; e < n; e += LY::kThreads) {
             const int i = list[e0 + e];
@@ -213,7 +215,7 @@ __global__ void __launch_bounds__(FwdLayout<PL>::kThreads) k_fwd(const float *__
                                                                  const int *__restrict__ ids,
                                                                  float *__restrict__ image,
                                                                  int *__restrict__ err) {
-    __shared__ FwdSmem<C> S;
+    __shared__ FwdSmem<C, kFwdBatch> S;
     const int b = blockIdx.x / g.T, t = blockIdx.x - b * g.T;
     const int ty = t / g.TX, tx = t - ty * g.TX;
     const int X0 = tx * kTile, Y0 = ty * kTile;
@@ -232,7 +234,7 @@ __global__ void __launch_bounds__(FwdLayout<PL>::kThreads) k_fwd(const float *__
 #pragma unroll
         for (int c = 0; c < C; ++c) amp[c] = pa[c];
     };
-    render_list<C, PL>(g, fetch, ids + L0, L1 - L0, X0, Y0, err, S, acc);
+    render_list<C, PL, kFwdBatch>(g, fetch, ids + L0, L1 - L0, X0, Y0, err, S, acc);
     store_tile<C, PL>(g, b, X0, Y0, image, acc);
 }
 
@@ -244,7 +246,7 @@ __global__ void __launch_bounds__(FwdLayout<PL>::kThreads) k_fwd_cluster(
     int *__restrict__ ids, float *__restrict__ image, int *__restrict__ err) {
     constexpr int NT = FwdLayout<PL>::kThreads;
     constexpr int NW = NT / 32;
-    __shared__ FwdSmem<C> S;
+    __shared__ FwdSmem<C, kClusterBatch> S;
     __shared__ int cnt[kClusterTiles];                 // this chunk's count per tile
     __shared__ int tab[kClusterTiles][kClusterTiles];  // tab[r][t] = count of chunk r in tile t
     __shared__ int base[kClusterTiles];                // next list slot of this chunk, per tile
@@ -384,7 +386,7 @@ __global__ void __launch_bounds__(FwdLayout<PL>::kThreads) k_fwd_cluster(
 #pragma unroll
             for (int c = 0; c < C; ++c) amp[c] = pa[c];
         };
-        render_list<C, PL>(g, fetch, src, L, X0, Y0, err, S, acc);
+        render_list<C, PL, kClusterBatch>(g, fetch, src, L, X0, Y0, err, S, acc);
     } else {
         auto fetch = [&](int i, float4 &A, float4 &Q, float (&amp)[C]) {
             const size_t gid = (size_t)b * g.N + i;
@@ -394,7 +396,7 @@ __global__ void __launch_bounds__(FwdLayout<PL>::kThreads) k_fwd_cluster(
 #pragma unroll
             for (int c = 0; c < C; ++c) amp[c] = pa[c];
         };
-        render_list<C, PL>(g, fetch, src, L, X0, Y0, err, S, acc);
+        render_list<C, PL, kClusterBatch>(g, fetch, src, L, X0, Y0, err, S, acc);
     }
     store_tile<C, PL>(g, b, X0, Y0, image, acc);
     if (onchip) cluster.sync();  // peers may still read this block's records
