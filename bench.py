@@ -282,22 +282,24 @@ class Step:
       split -- [event] forward [event] backward [event]    (stage times)
       fwd   -- [event] bins [event] forward from bins [event] (k_fwd alone)"""
 
-    def __init__(self, R, torch, w, seed, device):
+    def __init__(self, R, torch, w, seed, device, dtype=None):
         self.R, self.torch, self.w, self.device = R, torch, w, device
+        self.dtype = torch.float32 if dtype is None else dtype  # image / dL/dI storage
         p, g = make_inputs(w, seed)
         self.evals = in_grid_evals(p, w.H, w.W, w.k)
         self.h_params = torch.from_numpy(p).pin_memory()
         self.h_grad = torch.from_numpy(g).pin_memory()
         self.params = self.h_params.to(device)
-        self.grad = self.h_grad.to(device)
-        self.image = torch.empty((w.B, w.C, w.H, w.W), dtype=torch.float32, device=device)
+        self.grad = self.h_grad.to(device).to(self.dtype)
+        self.image = torch.empty((w.B, w.C, w.H, w.W), dtype=self.dtype, device=device)
         self.dparams = torch.empty_like(self.params)
         self.ws = R.Workspace.for_sizes(w.B, w.N, w.C, w.H, w.W, w.k, device)
         self.graphs, self.events = {}, {}
 
     def fwd(self, reuse_bins=False):
         w = self.w
-        self.R.render_fwd(self.params, w.H, w.W, w.k, self.ws, self.image, reuse_bins=reuse_bins)
+        self.R.render_fwd(self.params, w.H, w.W, w.k, self.ws, self.image, reuse_bins=reuse_bins,
+                          dtype=self.dtype)
 
     def bwd(self):
         w = self.w
@@ -612,6 +614,21 @@ def run_gpu(args, w):
             sweep[name]["loss_frac"] = lbs.entry(lms, peak_tops)["roofline"]["frac"]
             del lbs
 
+    # Reduced-precision storage of image and dL/dI (fp32 sums): the same step.
+    storage = {}
+    if rank == 0:
+        for dname in ("float16", "bfloat16"):
+            st = Step(R, torch, w, rank_seed(w, rank), device, dtype=getattr(torch, dname))
+            st.capture()
+            for _ in range(5):
+                flush.fill_(1)
+                st.replay()
+            pr = time_graph(st, "main", flush, args.sweep_steps, stream)
+            R.check_device_error(st.ws, device)
+            tot = float(pr[:, 0].mean())
+            storage[dname] = {"ms_per_step": tot, "evals_per_s": st.evals / (tot * 1e-3)}
+            del st
+
     knobs = {}
     if args.knobs and args.sweep and rank == 0:
         from differentiable_gaussian_splatting_pdr_b200.inputs import knob_workloads
@@ -666,6 +683,7 @@ def run_gpu(args, w):
             "loss_l1_ssim": loss_entry,
             "sweep": sweep,
             "knobs": knobs,
+            "storage_half": storage,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -40,6 +40,8 @@ SIGNATURES = {
     "pdr_check_device_error": (_i, [_vp, _vp]),
     "pdr_render_fwd_noalloc": (_i, [_vp] + [_i] * 6 + [_vp, _vp]),
     "pdr_loss_workspace_bytes": (_sz, [_i] * 4),
+    "pdr_render_fwd_ex": (_i, [_vp] + [_i] * 6 + [_vp, _i, _vp, _sz, _i, _vp]),
+    "pdr_render_bwd_ex": (_i, [_vp, _vp, _i] + [_i] * 6 + [_vp, _vp, _sz, _i, _vp]),
     "pdr_loss_l1_ssim": (_i, [_vp, _vp] + [_i] * 4 + [ctypes.c_float, ctypes.c_float] + [_vp] * 3 + [_sz, _vp]),
 }
 

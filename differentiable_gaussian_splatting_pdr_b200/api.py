@@ -84,25 +84,33 @@ def build_bins(params: torch.Tensor, H: int, W: int, k: int,
     return ws
 
 
+# Image storage types of the _ex entry points (pdr_dtype in include/pdr.h).
+_DTYPES = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
+
+
 def render_fwd(params: torch.Tensor, H: int, W: int, k: int, workspace: Workspace | None = None,
-               out: torch.Tensor | None = None, reuse_bins: bool = False):
+               out: torch.Tensor | None = None, reuse_bins: bool = False,
+               dtype: torch.dtype = torch.float32):
     """Forward render; returns (image [B, C, H, W], workspace holding the bins).
 
     reuse_bins=True renders from the bins already in `workspace` (built by
-    build_bins or an earlier call on the same params and sizes)."""
+    build_bins or an earlier call on the same params and sizes).  dtype
+    float16 / bfloat16 stores the image in that type (fp32 sums, rounded once)."""
     B, N, C = _check_params(params)
     dev = params.device
+    if dtype not in _DTYPES:
+        raise ValueError("dtype must be float32, float16 or bfloat16")
     holds = bool(reuse_bins and workspace is not None and workspace.shape == (B, N, C, H, W, k))
     ws = _workspace(workspace, B, N, C, H, W, k, dev)
     if ws is not workspace:
         holds = False
     if out is None:
-        out = torch.empty((B, C, H, W), dtype=torch.float32, device=dev)
-    elif out.shape != (B, C, H, W) or out.dtype != torch.float32 or not out.is_contiguous():
-        raise ValueError("out must be contiguous fp32 [B, C, H, W]")
+        out = torch.empty((B, C, H, W), dtype=dtype, device=dev)
+    elif out.shape != (B, C, H, W) or out.dtype != dtype or not out.is_contiguous():
+        raise ValueError("out must be contiguous %s [B, C, H, W]" % dtype)
     lib = _lib.load()
-    _lib.check("pdr_render_fwd", lib.pdr_render_fwd(
-        _ptr(params), B, N, C, H, W, k, _ptr(out), _ptr(ws.buf), ws.buf.numel(),
+    _lib.check("pdr_render_fwd_ex", lib.pdr_render_fwd_ex(
+        _ptr(params), B, N, C, H, W, k, _ptr(out), _DTYPES[dtype], _ptr(ws.buf), ws.buf.numel(),
         1 if holds else 0, _stream(dev)))
     ws.shape = (B, N, C, H, W, k)
     return out, ws
@@ -117,8 +125,8 @@ def render_bwd(params: torch.Tensor, grad_image: torch.Tensor, H: int, W: int, k
     `workspace`; otherwise (or without a matching workspace) they are rebuilt."""
     B, N, C = _check_params(params)
     dev = params.device
-    if grad_image.shape != (B, C, H, W) or grad_image.dtype != torch.float32 or not grad_image.is_cuda:
-        raise ValueError("grad_image must be fp32 CUDA [B, C, H, W]")
+    if grad_image.shape != (B, C, H, W) or grad_image.dtype not in _DTYPES or not grad_image.is_cuda:
+        raise ValueError("grad_image must be a float32 / float16 / bfloat16 CUDA [B, C, H, W]")
     grad_image = grad_image.contiguous()
     holds = bool(reuse_bins and workspace is not None and workspace.shape == (B, N, C, H, W, k))
     ws = _workspace(workspace, B, N, C, H, W, k, dev)
@@ -127,9 +135,9 @@ def render_bwd(params: torch.Tensor, grad_image: torch.Tensor, H: int, W: int, k
     if out is None:
         out = torch.empty_like(params)
     lib = _lib.load()
-    _lib.check("pdr_render_bwd", lib.pdr_render_bwd(
-        _ptr(params), _ptr(grad_image), B, N, C, H, W, k, _ptr(out), _ptr(ws.buf),
-        ws.buf.numel(), 1 if holds else 0, _stream(dev)))
+    _lib.check("pdr_render_bwd_ex", lib.pdr_render_bwd_ex(
+        _ptr(params), _ptr(grad_image), _DTYPES[grad_image.dtype], B, N, C, H, W, k, _ptr(out),
+        _ptr(ws.buf), ws.buf.numel(), 1 if holds else 0, _stream(dev)))
     ws.shape = (B, N, C, H, W, k)
     return out
 

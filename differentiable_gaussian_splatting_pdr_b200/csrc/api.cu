@@ -62,6 +62,7 @@ pdr_status make_geom(int B, int N, int C, int H, int W, int k, Geom *g) {
     g->fwd_pl = (long long)B * T <= 2368 ? 2 : 4;  // small grids: more, shorter lanes per tile
     g->out_vec2 = 0;
     g->out_vec4 = 0;
+    g->img_dtype = PDR_F32;
     return PDR_OK;
 }
 
@@ -149,18 +150,26 @@ pdr_status pdr_build_bins(const float *params, int B, int N, int C, int H, int W
     return from_cuda(bin(params, g, carve(workspace, L), static_cast<cudaStream_t>(stream)));
 }
 
-pdr_status pdr_render_fwd(const float *params, int B, int N, int C, int H, int W, int k,
-                          float *image, void *workspace, size_t workspace_bytes,
-                          int workspace_holds_bins, void *stream) {
+static bool dtype_ok(int dtype, const void *p) {
+    if (dtype == PDR_F32) return (reinterpret_cast<uintptr_t>(p) & 3) == 0;
+    if (dtype == PDR_F16 || dtype == PDR_BF16) return (reinterpret_cast<uintptr_t>(p) & 1) == 0;
+    return false;
+}
+
+pdr_status pdr_render_fwd_ex(const float *params, int B, int N, int C, int H, int W, int k,
+                             void *image, int image_dtype, void *workspace,
+                             size_t workspace_bytes, int workspace_holds_bins, void *stream) {
     Geom g;
     pdr_status st = make_geom(B, N, C, H, W, k, &g);
     if (st != PDR_OK) return st;
-    if (!params || !image || !aligned4(params) || !aligned4(image)) return PDR_ERR_INVALID_ARG;
+    if (!params || !image || !aligned4(params) || !dtype_ok(image_dtype, image))
+        return PDR_ERR_INVALID_ARG;
     Layout L;
     st = check_ws(g, workspace, workspace_bytes, &L);
     if (st != PDR_OK) return st;
     const Workspace ws = carve(workspace, L);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    g.img_dtype = image_dtype;
     g.out_vec2 = ((g.W & 1) == 0) && ((reinterpret_cast<uintptr_t>(image) & 7) == 0);
     g.out_vec4 = ((g.W & 3) == 0) && ((reinterpret_cast<uintptr_t>(image) & 15) == 0);
     if (!workspace_holds_bins && g.cluster_fwd)  // small frames: bins + render, one launch
@@ -172,26 +181,42 @@ pdr_status pdr_render_fwd(const float *params, int B, int N, int C, int H, int W
     return from_cuda(launch_fwd(params, g, ws, image, s, false));
 }
 
-pdr_status pdr_render_bwd(const float *params, const float *grad_image, int B, int N, int C,
-                          int H, int W, int k, float *grad_params, void *workspace,
-                          size_t workspace_bytes, int workspace_holds_fwd_bins,
-                          void *stream) {
+pdr_status pdr_render_fwd(const float *params, int B, int N, int C, int H, int W, int k,
+                          float *image, void *workspace, size_t workspace_bytes,
+                          int workspace_holds_bins, void *stream) {
+    return pdr_render_fwd_ex(params, B, N, C, H, W, k, image, PDR_F32, workspace, workspace_bytes,
+                             workspace_holds_bins, stream);
+}
+
+pdr_status pdr_render_bwd_ex(const float *params, const void *grad_image, int grad_dtype, int B,
+                             int N, int C, int H, int W, int k, float *grad_params,
+                             void *workspace, size_t workspace_bytes,
+                             int workspace_holds_fwd_bins, void *stream) {
     Geom g;
     pdr_status st = make_geom(B, N, C, H, W, k, &g);
     if (st != PDR_OK) return st;
-    if (!params || !grad_image || !grad_params || !aligned4(params) || !aligned4(grad_image) ||
-        !aligned4(grad_params))
+    if (!params || !grad_image || !grad_params || !aligned4(params) ||
+        !dtype_ok(grad_dtype, grad_image) || !aligned4(grad_params))
         return PDR_ERR_INVALID_ARG;
     Layout L;
     st = check_ws(g, workspace, workspace_bytes, &L);
     if (st != PDR_OK) return st;
     const Workspace ws = carve(workspace, L);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    g.img_dtype = grad_dtype;
     if (!workspace_holds_fwd_bins) {
         st = from_cuda(bin(params, g, ws, s));
         if (st != PDR_OK) return st;
     }
     return from_cuda(launch_bwd(params, grad_image, g, ws, grad_params, s));
+}
+
+pdr_status pdr_render_bwd(const float *params, const float *grad_image, int B, int N, int C,
+                          int H, int W, int k, float *grad_params, void *workspace,
+                          size_t workspace_bytes, int workspace_holds_fwd_bins,
+                          void *stream) {
+    return pdr_render_bwd_ex(params, grad_image, PDR_F32, B, N, C, H, W, k, grad_params,
+                             workspace, workspace_bytes, workspace_holds_fwd_bins, stream);
 }
 
 pdr_status pdr_bin(const float *params, int B, int N, int C, int H, int W, int k,

@@ -2,6 +2,8 @@
 // tile kernel, backward home-tile kernel).  Host API in api.cu.
 #pragma once
 
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -36,6 +38,7 @@ struct Geom {
     int fwd_pl;         // forward pixels per lane (2 or 4)
     int out_vec2;       // 1 if the output image allows 8-byte 2-pixel stores
     int out_vec4;       // 1 if the output image allows 16-byte 4-pixel stores
+    int img_dtype;      // storage of image / dL/dI: PDR_F32, PDR_F16 or PDR_BF16
 };
 
 constexpr int kBinChunk = 1024;        // Gaussians per binning block (large frames)
@@ -128,6 +131,22 @@ __device__ __forceinline__ int home_tile(int cx, int cy, const Geom &g) {
     return hy * g.TX + hx;
 }
 
+// One element of an image stored as fp32, fp16 or bf16 (dtype uniform per
+// launch), read or written as fp32.
+__device__ __forceinline__ float img_load(const void *p, size_t i, int dtype) {
+    if (dtype == 1) return __half2float(static_cast<const __half *>(p)[i]);
+    if (dtype == 2) return __bfloat162float(static_cast<const __nv_bfloat16 *>(p)[i]);
+    return static_cast<const float *>(p)[i];
+}
+__device__ __forceinline__ void img_store(void *p, size_t i, int dtype, float v) {
+    if (dtype == 1)
+        static_cast<__half *>(p)[i] = __float2half_rn(v);
+    else if (dtype == 2)
+        static_cast<__nv_bfloat16 *>(p)[i] = __float2bfloat16_rn(v);
+    else
+        static_cast<float *>(p)[i] = v;
+}
+
 // 2^x on the MUFU unit (flush-to-zero for results below the normal range).
 __device__ __forceinline__ float ex2(float x) {
     float y;
@@ -176,8 +195,8 @@ cudaError_t launch_bin(const float *params, const Geom &g, const Workspace &ws,
                        cudaStream_t s);
 // bin_inside: bin and render in one launch (g.cluster_fwd frames only).
 cudaError_t launch_fwd(const float *params, const Geom &g, const Workspace &ws,
-                       float *image, cudaStream_t s, bool bin_inside);
-cudaError_t launch_bwd(const float *params, const float *grad_image, const Geom &g,
+                       void *image, cudaStream_t s, bool bin_inside);
+cudaError_t launch_bwd(const float *params, const void *grad_image, const Geom &g,
                        const Workspace &ws, float *grad_params, cudaStream_t s);
 
 // Dynamic shared memory needed by the kernels for these sizes.

@@ -73,7 +73,7 @@ __device__ __forceinline__ void load_gpix(const float *gh, int pix, float (&gv)[
 
 template <int C, int KT>
 __global__ void __launch_bounds__(kBwdThreads) k_bwd(const float *__restrict__ params,
-                                                     const float *__restrict__ gimg, Geom g,
+                                                     const void *__restrict__ gimg, Geom g,
                                                      const float4 *__restrict__ gr,
                                                      const int *__restrict__ offs,
                                                      const int *__restrict__ ids,
@@ -148,7 +148,7 @@ __global__ void __launch_bounds__(kBwdThreads) k_bwd(const float *__restrict__ p
             const bool in = pix < RS * RS && core && x >= 0 && x < g.W && y >= 0 && y < g.H;
 #pragma unroll
             for (int c = 0; c < GP; ++c)
-                v[u][c] = (in && c < C) ? gimg[(((size_t)b * C + c) * g.H + y) * g.W + x] : 0.0f;
+                v[u][c] = (in && c < C) ? img_load(gimg, (((size_t)b * C + c) * g.H + y) * g.W + x, g.img_dtype) : 0.0f;
         }
 #pragma unroll
         for (int u = 0; u < kStageU; ++u) {
@@ -339,7 +339,7 @@ struct PairShape {
 
 template <int C, int K>
 __global__ void __launch_bounds__(kBwdThreads, 3) k_bwd_pairs(const float *__restrict__ params,
-                                                           const float *__restrict__ gimg, Geom g,
+                                                           const void *__restrict__ gimg, Geom g,
                                                            const float4 *__restrict__ gr,
                                                            const int *__restrict__ offs,
                                                            const int *__restrict__ ids,
@@ -391,7 +391,7 @@ __global__ void __launch_bounds__(kBwdThreads, 3) k_bwd_pairs(const float *__res
                 const bool in = rowin && x >= 0 && x < g.W && x <= X0 + kTile - 1 + R;
 #pragma unroll
                 for (int c = 0; c < 2 * NPL; ++c)
-                    v[u][q][c] = (in && c < C) ? gimg[(((size_t)b * C + c) * g.H + y) * g.W + x] : 0.0f;
+                    v[u][q][c] = (in && c < C) ? img_load(gimg, (((size_t)b * C + c) * g.H + y) * g.W + x, g.img_dtype) : 0.0f;
             }
         }
 #pragma unroll
@@ -569,9 +569,10 @@ __global__ void __launch_bounds__(kBwdThreads, 3) k_bwd_pairs(const float *__res
                     for (int c = 0; c < 2 * NPL; ++c) {
                         float lo = 0.0f, hi = 0.0f;
                         if (c < C && y >= 0 && y < g.H) {
-                            const float *rowp = gimg + (((size_t)b * C + c) * g.H + y) * g.W;
-                            if (x >= 0 && x < g.W) lo = rowp[x];
-                            if (x + 1 >= 0 && x + 1 < g.W && pc < NPW - 1) hi = rowp[x + 1];
+                            const size_t row = (((size_t)b * C + c) * g.H + y) * g.W;
+                            if (x >= 0 && x < g.W) lo = img_load(gimg, row + x, g.img_dtype);
+                            if (x + 1 >= 0 && x + 1 < g.W && pc < NPW - 1)
+                                hi = img_load(gimg, row + x + 1, g.img_dtype);
                         }
                         gc[c] = make_float2(lo, hi);
                     }
@@ -623,7 +624,7 @@ __global__ void __launch_bounds__(kBwdThreads, 3) k_bwd_pairs(const float *__res
 }
 
 template <int C, int K>
-cudaError_t launch_bwd_pairs(const float *params, const float *grad_image, const Geom &g,
+cudaError_t launch_bwd_pairs(const float *params, const void *grad_image, const Geom &g,
                              const Workspace &ws, float *grad_params, cudaStream_t s) {
     constexpr size_t smem = PairShape<C, K>::SMEM;
     static_assert(smem <= 200 * 1024, "staged dL/dI does not fit");
@@ -638,7 +639,7 @@ cudaError_t launch_bwd_pairs(const float *params, const float *grad_image, const
 }
 
 template <int C, int KT>
-cudaError_t launch_bwd_ck(const float *params, const float *grad_image, const Geom &g,
+cudaError_t launch_bwd_ck(const float *params, const void *grad_image, const Geom &g,
                           const Workspace &ws, float *grad_params, cudaStream_t s) {
     const size_t smem = bwd_smem(g);
     if (smem > 48 * 1024) {
@@ -652,7 +653,7 @@ cudaError_t launch_bwd_ck(const float *params, const float *grad_image, const Ge
 }
 
 template <int C>
-cudaError_t launch_bwd_c(const float *params, const float *grad_image, const Geom &g,
+cudaError_t launch_bwd_c(const float *params, const void *grad_image, const Geom &g,
                          const Workspace &ws, float *grad_params, cudaStream_t s) {
     // Measured on B200: the pixel-pair kernel pays off for wide windows
     // (k >= 13); for smaller windows the per-Gaussian work is short and the
@@ -682,7 +683,7 @@ size_t bwd_smem(const Geom &g) {
            sizeof(float) * (size_t)RS * RP * GP;
 }
 
-cudaError_t launch_bwd(const float *params, const float *grad_image, const Geom &g,
+cudaError_t launch_bwd(const float *params, const void *grad_image, const Geom &g,
                        const Workspace &ws, float *grad_params, cudaStream_t s) {
     switch (g.C) {
         case 1: return launch_bwd_c<1>(params, grad_image, g, ws, grad_params, s);

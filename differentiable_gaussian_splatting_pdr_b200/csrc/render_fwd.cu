@@ -183,13 +183,24 @@ __device__ __forceinline__ void render_list(const Geom &g, Fetch fetch, const in
 
 template <int C, int PL>
 __device__ __forceinline__ void store_tile(const Geom &g, int b, int X0, int Y0,
-                                           float *__restrict__ image, const float (&acc)[PL][C]) {
+                                           void *__restrict__ image_, const float (&acc)[PL][C]) {
     using LY = FwdLayout<PL>;
     const int tid = threadIdx.x;
     const int grp = tid / LY::kLanes, lig = tid % LY::kLanes;
     const int lrow = lig / (4 / PL), lcol = (lig % (4 / PL)) * PL;
     const int x = X0 + 4 * (grp & 3) + lcol, y = Y0 + 4 * (grp >> 2) + lrow;
     if (y >= g.H) return;
+    if (g.img_dtype != 0) {  // fp16 / bf16 storage: fp32 sums, rounded to nearest once
+#pragma unroll
+        for (int c = 0; c < C; ++c) {
+            const size_t o = (((size_t)b * C + c) * g.H + y) * g.W + x;
+#pragma unroll
+            for (int j = 0; j < PL; ++j)
+                if (x + j < g.W) img_store(image_, o + j, g.img_dtype, acc[j][c]);
+        }
+        return;
+    }
+    float *image = static_cast<float *>(image_);
     const bool vec = (x + PL - 1 < g.W) && (PL == 4 ? g.out_vec4 : g.out_vec2);
 #pragma unroll
     for (int c = 0; c < C; ++c) {
@@ -213,7 +224,7 @@ __global__ void __launch_bounds__(FwdLayout<PL>::kThreads) k_fwd(const float *__
                                                                  const float4 *__restrict__ gr,
                                                                  const int *__restrict__ offs,
                                                                  const int *__restrict__ ids,
-                                                                 float *__restrict__ image,
+                                                                 void *__restrict__ image,
                                                                  int *__restrict__ err) {
     __shared__ FwdSmem<C, kFwdBatch> S;
     const int b = blockIdx.x / g.T, t = blockIdx.x - b * g.T;
@@ -243,7 +254,7 @@ __global__ void __launch_bounds__(FwdLayout<PL>::kThreads) k_fwd(const float *__
 template <int C, int PL>
 __global__ void __launch_bounds__(FwdLayout<PL>::kThreads) k_fwd_cluster(
     const float *__restrict__ params, Geom g, float4 *__restrict__ gr, int *__restrict__ offs,
-    int *__restrict__ ids, float *__restrict__ image, int *__restrict__ err) {
+    int *__restrict__ ids, void *__restrict__ image, int *__restrict__ err) {
     constexpr int NT = FwdLayout<PL>::kThreads;
     constexpr int NW = NT / 32;
     __shared__ FwdSmem<C, kClusterBatch> S;
@@ -404,7 +415,7 @@ __global__ void __launch_bounds__(FwdLayout<PL>::kThreads) k_fwd_cluster(
 
 template <int C, int PL>
 cudaError_t launch_fwd_cluster(const float *params, const Geom &g, const Workspace &ws,
-                               float *image, cudaStream_t s) {
+                               void *image, cudaStream_t s) {
         cudaError_t e;
         if (g.T > 8) {
             e = cudaFuncSetAttribute(k_fwd_cluster<C, PL>,
@@ -430,7 +441,7 @@ cudaError_t launch_fwd_cluster(const float *params, const Geom &g, const Workspa
 }
 
 template <int C>
-cudaError_t launch_fwd_c(const float *params, const Geom &g, const Workspace &ws, float *image,
+cudaError_t launch_fwd_c(const float *params, const Geom &g, const Workspace &ws, void *image,
                          cudaStream_t s, bool bin_inside) {
     if (bin_inside)
         return g.fwd_pl == 2 ? launch_fwd_cluster<C, 2>(params, g, ws, image, s)
@@ -446,7 +457,7 @@ cudaError_t launch_fwd_c(const float *params, const Geom &g, const Workspace &ws
 
 }  // namespace
 
-cudaError_t launch_fwd(const float *params, const Geom &g, const Workspace &ws, float *image,
+cudaError_t launch_fwd(const float *params, const Geom &g, const Workspace &ws, void *image,
                        cudaStream_t s, bool bin_inside) {
     switch (g.C) {
         case 1: return launch_fwd_c<1>(params, g, ws, image, s, bin_inside);

@@ -175,6 +175,31 @@ pdr_status pdr_step_host(const float *h_params, const float *h_grad_image,
 pdr_status pdr_render_fwd_noalloc(const float *params, int B, int N, int C, int H,
                                   int W, int k, float *image, void *stream);
 
+/* ---- Reduced-precision image storage ------------------------------------------
+ * Image and dL/dI stored as fp16 or bf16 (half the bytes of the two largest
+ * tensors), every sum still in fp32: the forward rounds each pixel's fp32
+ * total to the storage type once (round to nearest even), the backward
+ * widens each dL/dI element to fp32 on load.  Motivated by the mixed-precision
+ * study of the hardware-rasterizer page ("contour-based differentiable
+ * rendering"); params and grad_params stay fp32 (small, and mu feeds the
+ * exact window centre).  The fp16/bf16 image of pdr_render_fwd_ex equals the
+ * fp32 image of pdr_render_fwd rounded to that type. */
+typedef enum { PDR_F32 = 0, PDR_F16 = 1, PDR_BF16 = 2 } pdr_dtype;
+
+/* pdr_render_fwd with the image stored as image_dtype (a pdr_dtype; the
+ * image pointer aligned to its element size).  pdr_render_fwd(...) is
+ * pdr_render_fwd_ex(..., image, PDR_F32, ...).  An unknown dtype returns
+ * PDR_ERR_INVALID_ARG. */
+pdr_status pdr_render_fwd_ex(const float *params, int B, int N, int C, int H, int W, int k,
+                             void *image, int image_dtype, void *workspace,
+                             size_t workspace_bytes, int workspace_holds_bins, void *stream);
+
+/* pdr_render_bwd with dL/dI stored as grad_dtype (a pdr_dtype). */
+pdr_status pdr_render_bwd_ex(const float *params, const void *grad_image, int grad_dtype, int B,
+                             int N, int C, int H, int W, int k, float *grad_params,
+                             void *workspace, size_t workspace_bytes,
+                             int workspace_holds_fwd_bins, void *stream);
+
 /* Synchronises `stream` and reports the device-side error word in the
  * workspace (PDR_ERR_INTERNAL if a kernel's own bounds check fired), then
  * clears it. */

@@ -251,3 +251,31 @@ def test_knob_workloads(name):
     w = knob_workloads()[name]
     p, g = make_inputs(w)
     check_all(p, g, w.H, w.W, w.k)
+
+
+@pytest.mark.parametrize("dtype,bar", [("float16", 1e-3), ("bfloat16", 8e-3)])
+@pytest.mark.parametrize("name", ["mono64", "rgb128", "field32x64"])
+def test_reduced_precision_storage(name, dtype, bar):
+    """Image and dL/dI stored as fp16 / bf16, sums in fp32: the stored image is
+    the fp32 image rounded once; gradients from a half-precision dL/dI match the
+    oracle given the same (widened) values at the fp32 bar."""
+    import torch
+    from differentiable_gaussian_splatting_pdr_b200 import api as R
+    tdt = getattr(torch, dtype)
+    w = WORKLOADS[name]
+    p, g = make_inputs(w)
+    dev = torch.device("cuda:0")
+    pt = torch.from_numpy(p).to(dev)
+    img32, ws = R.render_fwd(pt, w.H, w.W, w.k)
+    imgh, _ = R.render_fwd(pt, w.H, w.W, w.k, ws, reuse_bins=True, dtype=tdt)
+    torch.cuda.synchronize()
+    assert imgh.dtype == tdt
+    assert torch.equal(imgh, img32.to(tdt))  # rounded once, to nearest
+    ref = oracle.render_fwd(p, w.H, w.W, w.k)
+    assert fwd_err(imgh.float().cpu().numpy(), ref) <= bar
+    gh = torch.from_numpy(g).to(dev).to(tdt)
+    dp = R.render_bwd(pt, gh, w.H, w.W, w.k, ws, reuse_bins=True)
+    torch.cuda.synchronize()
+    gw = gh.float().cpu().numpy()
+    rdp = oracle.render_bwd(p, gw, w.H, w.W, w.k)
+    assert bwd_err(dp.cpu().numpy(), rdp) <= 1e-4
