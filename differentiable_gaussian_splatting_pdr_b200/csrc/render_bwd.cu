@@ -255,22 +255,44 @@ __global__ void __launch_bounds__(kBwdThreads) k_bwd(const float *__restrict__ p
             }
             if (lig < tail) eval(full);
 
-            // Fixed xor tree over the lanes of the group.
+            // The chain rule is linear in the sums, so each lane applies it to
+            // its own partial sums; a transposing xor tree then leaves lane j
+            // of the group with gradient component j (j < 8), summed over the
+            // group in a fixed order; components 8.. (C > 3) use a plain tree.
+            // 2 sinh(s1 - s2) = e^{d} - e^{-d}, via the base-2 exponential.
+            const float dl = (pp[2] - pp[3]) * 1.44269504088896340736f;
+            const float sh2 = kTwoLn2 * (ex2(dl) - ex2(-dl));
+            float v[8];
+            v[0] = kTwoLn2 * fmaf(a1, acc[0], a2 * acc[1]);  // dL/dmu_x
+            v[1] = kTwoLn2 * fmaf(b1, acc[0], b2 * acc[1]);  // dL/dmu_y
+            v[2] = kTwoLn2 * acc[2];                         // dL/ds_1
+            v[3] = kTwoLn2 * acc[4];                         // dL/ds_2
+            v[4] = sh2 * acc[3];                             // dL/dtheta
 #pragma unroll
-            for (int d = 1; d < kGroup; d <<= 1) {
+            for (int j = 5; j < 8; ++j) v[j] = j < NV ? acc[j < NV ? j : 0] : 0.0f;
+            const bool h2 = lig & 4, h1 = lig & 2, h0 = lig & 1;
 #pragma unroll
-                for (int j = 0; j < NV; ++j) acc[j] += __shfl_xor_sync(gmask, acc[j], d);
+            for (int i = 0; i < 4; ++i) {
+                const float send = h2 ? v[i] : v[i + 4], keep = h2 ? v[i + 4] : v[i];
+                v[i] = keep + __shfl_xor_sync(gmask, send, 4);
             }
-            if (lig == 0) {
-                const float s1 = pp[2], s2 = pp[3];
-                float *d = dparams + gid * g.P;
-                d[0] = kTwoLn2 * fmaf(a1, acc[0], a2 * acc[1]);
-                d[1] = kTwoLn2 * fmaf(b1, acc[0], b2 * acc[1]);
-                d[2] = kTwoLn2 * acc[2];
-                d[3] = kTwoLn2 * acc[4];
-                d[4] = kTwoLn2 * 2.0f * sinhf(s1 - s2) * acc[3];
 #pragma unroll
-                for (int c = 0; c < C; ++c) d[5 + c] = acc[5 + c];
+            for (int i = 0; i < 2; ++i) {
+                const float send = h1 ? v[i] : v[i + 2], keep = h1 ? v[i + 2] : v[i];
+                v[i] = keep + __shfl_xor_sync(gmask, send, 2);
+            }
+            {
+                const float send = h0 ? v[0] : v[1], keep = h0 ? v[1] : v[0];
+                v[0] = keep + __shfl_xor_sync(gmask, send, 1);
+            }
+            float *d = dparams + gid * g.P;
+            if (lig < NV) d[lig] = v[0];
+#pragma unroll
+            for (int j = 8; j < NV; ++j) {
+                float e = acc[j];
+#pragma unroll
+                for (int dd = 1; dd < kGroup; dd <<= 1) e += __shfl_xor_sync(gmask, e, dd);
+                if (lig == 0) d[j] = e;
             }
         }
         nh = 0;
