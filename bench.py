@@ -83,7 +83,8 @@ def source_hash(*names) -> str:
 
 KERNEL_SOURCES = {"k_fwd": ("render_fwd.cu", "common.cuh"),
                   "k_fwd_cluster": ("render_fwd.cu", "common.cuh"),
-                  "k_bwd": ("render_bwd.cu", "common.cuh")}
+                  "k_bwd": ("render_bwd.cu", "common.cuh"),
+                  "k_loss_tile": ("loss.cu", "common.cuh")}
 CLUSTER_MAX_TILES = 16       # frames of at most this many tiles ...
 CLUSTER_MAX_BLOCKS = 4 * 148  # ... in launches of at most this many blocks: k_fwd_cluster
 
@@ -409,6 +410,7 @@ class LossBench:
     CUDA events, L2 flushed before every call."""
 
     def __init__(self, R, torch, w, seed, device):
+        self.workload = w.name
         rng = np.random.default_rng(seed + 7)
         x = rng.uniform(0, 1, (w.B, w.C, w.H, w.W)).astype(np.float32)
         y = np.clip(x + rng.normal(0, 0.1, x.shape), 0, 1).astype(np.float32)
@@ -448,6 +450,7 @@ class LossBench:
                 "roofline": {"bound": "alu", "kernel": "k_loss_tile", "achieved": achieved,
                              "peak": peak_tops, "unit": "Tinst/s", "frac": achieved / peak_tops,
                              "ops_per_px": LOSS_OPS_PER_PX,
+                             "traffic": profiled_traffic("k_loss_tile", self.workload),
                              "algorithmic_bytes": 12 * self.px},
                 "data": "image ~ U[0,1], target = clip(image + N(0, 0.1)), lam 0.2"}
 
