@@ -6,20 +6,28 @@
 //   SSIM per (frame, channel) image with an 11 x 11 Gaussian window (sigma
 //   1.5), zero padding, C1 = (0.01 range)^2, C2 = (0.03 range)^2.
 //
-// k_loss_tile: one block per 32 x 32 output tile of one image.  The image and
-// the target are staged with a 10-pixel apron, shifted by a per-block
-// constant (the value at the tile centre): SSIM and its gradient are
-// invariant under that shift, and it keeps the fp32 variances and the final
-// gradient combination free of large cancellations.  Five separable window
-// sums (horizontal then vertical) give the moments mu_x, mu_y, E xx, E yy,
-// E xy on the tile plus a 5-pixel apron; there the SSIM map S and the
-// gradient coefficients
-//   A = dS/dmu_x - 2 mu_x dS/ds_xx - mu_y dS/ds_xy,  B = dS/ds_xx,  Cxy = dS/ds_xy
-// are formed (zero outside the image), and three more separable window sums
-// give dS_mean/dI = (G*A + 2 I (G*B) + T (G*Cxy)) / n on the tile.  Each block
-// leaves its partial sums of |I - T| and S in the workspace; k_loss_final
-// adds them in block order (fp64) into the loss.  Fixed order throughout:
-// bitwise reproducible.
+// Two tile kernels, one block per 32 x 32 tile of one (frame, channel)
+// image, and a final reduction:
+//   k_loss_coef  stages image and target with a 5-pixel apron, forms the five
+//                window moments mu_x, mu_y, E xx, E yy, E xy on the tile by
+//                separable sums (horizontal over the apron rows, then
+//                vertical), the SSIM map S and the gradient coefficients
+//                A = dS/dmu_x - 2 mu_x dS/ds_xx - mu_y dS/ds_xy,
+//                B = dS/ds_xx,  Cxy = dS/ds_xy
+//                (written to the workspace), and the tile's sums of |I - T|
+//                and S;
+//   k_loss_grad  stages A, B, Cxy with a 5-pixel apron (zero outside the
+//                image) and forms dS_mean/dI = (G*A + 2 I (G*B) + T (G*Cxy)) / n
+//                by separable sums, then dL/dI;
+//   k_loss_final adds the per-block sums in block order (fp64) into L.
+// Image and target are shifted by their values at the image centre: SSIM and
+// its gradient are invariant under the shift (A is formed with the shifted
+// means, the final combination with the shifted values: the shift cancels
+// pixel pair by pixel pair), and it keeps the fp32 variances and the final
+// combination free of large cancellations.  Taps come from the constant bank
+// (a kernel argument); each separable pass is register-blocked (a thread
+// produces RB neighbouring outputs from one streamed read of RB + 10
+// inputs).  Fixed order throughout: bitwise reproducible.
 #include <math.h>
 #include <stdint.h>
 
@@ -29,67 +37,70 @@
 namespace pdr {
 namespace {
 
-constexpr int kLT = 32;             // output tile edge
+constexpr int kLT = 32;             // tile edge
 constexpr int kLR = 5;              // window radius
 constexpr int kLW = 2 * kLR + 1;    // window taps
-constexpr int kLS = kLT + 2 * kLR;  // moment region edge (42)
-constexpr int kLI = kLT + 4 * kLR;  // staged input edge (52)
-constexpr int kLossThreads = 512;
-constexpr int kLU = (kLI * kLI + kLossThreads - 1) / kLossThreads;  // staged pixels per thread
+constexpr int kLS = kLT + 2 * kLR;  // tile plus apron (42)
+constexpr int kLossThreads = 256;
+constexpr int kLU = (kLS * kLS + kLossThreads - 1) / kLossThreads;  // staged pixels per thread
+constexpr int kRBH = 4;  // horizontal passes: 32 = 8 x 4 outputs per row
+constexpr int kRBV = 2;  // vertical passes:   32 = 16 x 2 outputs per column
 
-struct LossSmem {
-    float x[kLI][kLI];            // shifted image, zero-padded
-    float y[kLI][kLI];            // shifted target
-    float h[5][kLI][kLS];         // horizontal window sums (reused for the gradient pass)
-    float abc[3][kLS][kLS];       // A, B, Cxy on the tile and its apron
-    signed char sgn[kLT][kLT];    // sign(I - T) on the tile
-    float red[2][kLossThreads / 32];
-};
-
-// The window taps travel as a kernel argument (constant bank): every FMA
-// reads its tap without a shared-memory load.
+// The window taps travel as a kernel argument (constant bank).
 struct Taps {
     float t[kLW];
 };
 
-// Register-blocked passes: a thread produces RB neighbouring outputs of a
-// window sum from one streamed read of the RB + 10 inputs they share.
-constexpr int kRB2 = 6;  // horizontal moments: 42 = 7 x 6 outputs per row
-constexpr int kRB3 = 3;  // vertical moments:   42 = 14 x 3 outputs per column
-constexpr int kRB4 = 4;  // horizontal coefficients: 32 = 8 x 4
-constexpr int kRB5 = 2;  // vertical coefficients:   32 = 16 x 2
+struct CoefSmem {
+    float x[kLS][kLS];      // shifted image over the tile and its apron, zero-padded
+    float y[kLS][kLS];      // shifted target
+    float h[5][kLS][kLT];   // horizontal window sums of x, y, xx, yy, xy
+    float red[2][kLossThreads / 32];
+};
+struct GradSmem {
+    float abc[3][kLS][kLS];  // A, B, Cxy over the tile and its apron
+    float h[3][kLS][kLT];    // their horizontal window sums
+};
 
-__global__ void __launch_bounds__(kLossThreads) k_loss_tile(
-    const float *__restrict__ img, const float *__restrict__ tgt, int BC, int H, int W, int TX,
-    int TY, float lam, float C1, float C2, double inv_n, const Taps tp_,
-    float *__restrict__ grad, float *__restrict__ part) {
-    extern __shared__ float4 lsm4[];
-    LossSmem &S = *reinterpret_cast<LossSmem *>(lsm4);
-    const int tid = threadIdx.x;
+struct LossTile {
+    int im, X0, Y0;
+    size_t base;
+};
+__device__ __forceinline__ LossTile loss_tile(int W, int H, int TX, int TY) {
     const int tiles = TX * TY;
-    const int im = blockIdx.x / tiles, t = blockIdx.x - im * tiles;
-    const int ty = t / TX, tx = t - ty * TX;
-    const int X0 = tx * kLT, Y0 = ty * kLT;
-    const size_t base = (size_t)im * H * W;
-    const float *ip = img + base, *tp = tgt + base;
+    LossTile L;
+    L.im = blockIdx.x / tiles;
+    const int t = blockIdx.x - L.im * tiles;
+    const int ty = t / TX;
+    L.X0 = (t - ty * TX) * kLT;
+    L.Y0 = ty * kLT;
+    L.base = (size_t)L.im * H * W;
+    return L;
+}
+
+__global__ void __launch_bounds__(kLossThreads) k_loss_coef(
+    const float *__restrict__ img, const float *__restrict__ tgt, int H, int W, int TX, int TY,
+    float C1, float C2, const Taps tp_, float *__restrict__ coef, size_t n,
+    float *__restrict__ part) {
+    extern __shared__ float4 lsm4[];
+    CoefSmem &S = *reinterpret_cast<CoefSmem *>(lsm4);
+    const int tid = threadIdx.x;
+    const LossTile T = loss_tile(W, H, TX, TY);
+    const float *ip = img + T.base, *tp = tgt + T.base;
     const float *g = tp_.t;
+    const size_t mid = (size_t)(H / 2) * W + W / 2;  // the image's shift
+    const float sx = ip[mid], sy = tp[mid];
 
-    // Shift: the values at the tile centre (clamped into the image).
-    const int cyy = min(Y0 + kLT / 2, H - 1), cxx = min(X0 + kLT / 2, W - 1);
-    const float sx = ip[(size_t)cyy * W + cxx], sy = tp[(size_t)cyy * W + cxx];
-
-    // 1. stage the shifted inputs over [Y0 - 10, Y0 + 41] x [X0 - 10, X0 + 41]
-    //    (all of a thread's loads in flight together); the L1 term of the
-    //    tile's own pixels is taken from the unshifted values here.
+    // 1. stage [Y0 - 5, Y0 + 36] x [X0 - 5, X0 + 36]; |I - T| of the tile's pixels
     float lsum = 0.0f;
     {
         float xv[kLU], yv[kLU];
 #pragma unroll
         for (int u = 0; u < kLU; ++u) {
             const int i = u * kLossThreads + tid;
-            const int r = i / kLI, c = i - r * kLI;
-            const int y = Y0 - 2 * kLR + r, x = X0 - 2 * kLR + c;
-            const bool in = i < kLI * kLI && y >= 0 && y < H && x >= 0 && x < W;
+            const int r = i / kLS, c = i - r * kLS;
+            const int y = T.Y0 - kLR + r, x = T.X0 - kLR + c;
+            const bool in = i < kLS * kLS && y >= 0 && y < H && x >= 0 && x < W;
             const size_t o = in ? (size_t)y * W + x : 0;
             xv[u] = in ? ip[o] : 0.0f;
             yv[u] = in ? tp[o] : 0.0f;
@@ -97,35 +108,32 @@ __global__ void __launch_bounds__(kLossThreads) k_loss_tile(
 #pragma unroll
         for (int u = 0; u < kLU; ++u) {
             const int i = u * kLossThreads + tid;
-            if (i >= kLI * kLI) continue;
-            const int r = i / kLI, c = i - r * kLI;
+            if (i >= kLS * kLS) continue;
+            const int r = i / kLS, c = i - r * kLS;
             S.x[r][c] = xv[u] - sx;
             S.y[r][c] = yv[u] - sy;
-            const int tr = r - 2 * kLR, tc = c - 2 * kLR;
-            if (tr >= 0 && tr < kLT && tc >= 0 && tc < kLT) {
-                const float diff = xv[u] - yv[u];  // unshifted: ties stay exact zeros
-                S.sgn[tr][tc] = diff > 0.0f ? 1 : (diff < 0.0f ? -1 : 0);
-                if (Y0 + tr < H && X0 + tc < W) lsum += fabsf(diff);
-            }
+            const int tr = r - kLR, tc = c - kLR;
+            if (tr >= 0 && tr < kLT && tc >= 0 && tc < kLT && T.Y0 + tr < H && T.X0 + tc < W)
+                lsum += fabsf(xv[u] - yv[u]);
         }
     }
     __syncthreads();
 
-    // 2. horizontal window sums of x, y, xx, yy, xy over all staged rows
-    for (int it = tid; it < kLI * (kLS / kRB2); it += kLossThreads) {
-        const int r = it / (kLS / kRB2), c0 = (it - r * (kLS / kRB2)) * kRB2;
-        float m[5][kRB2];
+    // 2. horizontal sums of x, y, xx, yy, xy (all staged rows, the tile's columns)
+    for (int it = tid; it < kLS * (kLT / kRBH); it += kLossThreads) {
+        const int r = it / (kLT / kRBH), c0 = (it - r * (kLT / kRBH)) * kRBH;
+        float m[5][kRBH];
 #pragma unroll
-        for (int j = 0; j < kRB2; ++j)
+        for (int j = 0; j < kRBH; ++j)
 #pragma unroll
             for (int q = 0; q < 5; ++q) m[q][j] = 0.0f;
 #pragma unroll
-        for (int k = 0; k < kRB2 + kLW - 1; ++k) {
+        for (int k = 0; k < kRBH + kLW - 1; ++k) {
             const float a = S.x[r][c0 + k], b = S.y[r][c0 + k];
             const float aa = a * a, bb = b * b, ab = a * b;
 #pragma unroll
-            for (int j = 0; j < kRB2; ++j) {
-                const int d = k - j;  // tap of output c0 + j
+            for (int j = 0; j < kRBH; ++j) {
+                const int d = k - j;
                 if (d < 0 || d >= kLW) continue;
                 m[0][j] = fmaf(g[d], a, m[0][j]);
                 m[1][j] = fmaf(g[d], b, m[1][j]);
@@ -137,26 +145,26 @@ __global__ void __launch_bounds__(kLossThreads) k_loss_tile(
 #pragma unroll
         for (int q = 0; q < 5; ++q)
 #pragma unroll
-            for (int j = 0; j < kRB2; ++j) S.h[q][r][c0 + j] = m[q][j];
+            for (int j = 0; j < kRBH; ++j) S.h[q][r][c0 + j] = m[q][j];
     }
     __syncthreads();
 
-    // 3. vertical sums -> moments; SSIM map and gradient coefficients
+    // 3. vertical sums -> moments on the tile; SSIM and the coefficients
     float ssum = 0.0f;
-    for (int it = tid; it < (kLS / kRB3) * kLS; it += kLossThreads) {
-        const int rb = it / kLS, c = it - rb * kLS, r0 = rb * kRB3;
-        float m[5][kRB3];
+    for (int it = tid; it < (kLT / kRBV) * kLT; it += kLossThreads) {
+        const int rb = it / kLT, c = it - rb * kLT, r0 = rb * kRBV;
+        float m[5][kRBV];
 #pragma unroll
-        for (int j = 0; j < kRB3; ++j)
+        for (int j = 0; j < kRBV; ++j)
 #pragma unroll
             for (int q = 0; q < 5; ++q) m[q][j] = 0.0f;
 #pragma unroll
-        for (int k = 0; k < kRB3 + kLW - 1; ++k) {
+        for (int k = 0; k < kRBV + kLW - 1; ++k) {
             float v[5];
 #pragma unroll
             for (int q = 0; q < 5; ++q) v[q] = S.h[q][r0 + k][c];
 #pragma unroll
-            for (int j = 0; j < kRB3; ++j) {
+            for (int j = 0; j < kRBV; ++j) {
                 const int d = k - j;
                 if (d < 0 || d >= kLW) continue;
 #pragma unroll
@@ -164,94 +172,28 @@ __global__ void __launch_bounds__(kLossThreads) k_loss_tile(
             }
         }
 #pragma unroll
-        for (int j = 0; j < kRB3; ++j) {
-            const int r = r0 + j;
-            const int y = Y0 - kLR + r, x = X0 - kLR + c;
-            float A = 0.f, Bc = 0.f, Cc = 0.f;
-            if (y >= 0 && y < H && x >= 0 && x < W) {
-                const float mx = m[0][j], my = m[1][j];  // shifted means
-                const float vxx = fmaf(-mx, mx, m[2][j]), vyy = fmaf(-my, my, m[3][j]);
-                const float vxy = fmaf(-mx, my, m[4][j]);
-                const float ux = mx + sx, uy = my + sy;  // true means
-                const float N1 = fmaf(2.0f * ux, uy, C1), N2 = fmaf(2.0f, vxy, C2);
-                const float D1 = fmaf(ux, ux, fmaf(uy, uy, C1)), D2 = vxx + vyy + C2;
-                const float rD1 = 1.0f / D1, rD2 = 1.0f / D2, rD = rD1 * rD2;
-                const float s = N1 * N2 * rD;
-                const float dmu = 2.0f * uy * N2 * rD - 2.0f * ux * s * rD1;
-                Bc = -s * rD2;
-                Cc = 2.0f * N1 * rD;
-                A = dmu - 2.0f * mx * Bc - my * Cc;  // shifted means: the shift cancels exactly
-                if (r >= kLR && r < kLR + kLT && c >= kLR && c < kLR + kLT) ssum += s;
-            }
-            S.abc[0][r][c] = A;
-            S.abc[1][r][c] = Bc;
-            S.abc[2][r][c] = Cc;
-        }
-    }
-    __syncthreads();
-
-    // 4. horizontal window sums of A, B, Cxy over the moment rows
-    for (int it = tid; it < kLS * (kLT / kRB4); it += kLossThreads) {
-        const int r = it / (kLT / kRB4), c0 = (it - r * (kLT / kRB4)) * kRB4;
-        float m[3][kRB4];
-#pragma unroll
-        for (int j = 0; j < kRB4; ++j)
-#pragma unroll
-            for (int q = 0; q < 3; ++q) m[q][j] = 0.0f;
-#pragma unroll
-        for (int k = 0; k < kRB4 + kLW - 1; ++k) {
-            float v[3];
-#pragma unroll
-            for (int q = 0; q < 3; ++q) v[q] = S.abc[q][r][c0 + k];
-#pragma unroll
-            for (int j = 0; j < kRB4; ++j) {
-                const int d = k - j;
-                if (d < 0 || d >= kLW) continue;
-#pragma unroll
-                for (int q = 0; q < 3; ++q) m[q][j] = fmaf(g[d], v[q], m[q][j]);
-            }
-        }
-#pragma unroll
-        for (int q = 0; q < 3; ++q)
-#pragma unroll
-            for (int j = 0; j < kRB4; ++j) S.h[q][r][c0 + j] = m[q][j];
-    }
-    __syncthreads();
-
-    // 5. vertical sums -> dL/dI on the tile
-    const float wl1 = (float)((1.0 - (double)lam) * inv_n), wss = (float)((double)lam * inv_n);
-    for (int it = tid; it < (kLT / kRB5) * kLT; it += kLossThreads) {
-        const int rb = it / kLT, c = it - rb * kLT, r0 = rb * kRB5;
-        float m[3][kRB5];
-#pragma unroll
-        for (int j = 0; j < kRB5; ++j)
-#pragma unroll
-            for (int q = 0; q < 3; ++q) m[q][j] = 0.0f;
-#pragma unroll
-        for (int k = 0; k < kRB5 + kLW - 1; ++k) {
-            float v[3];
-#pragma unroll
-            for (int q = 0; q < 3; ++q) v[q] = S.h[q][r0 + k][c];
-#pragma unroll
-            for (int j = 0; j < kRB5; ++j) {
-                const int d = k - j;
-                if (d < 0 || d >= kLW) continue;
-#pragma unroll
-                for (int q = 0; q < 3; ++q) m[q][j] = fmaf(g[d], v[q], m[q][j]);
-            }
-        }
-#pragma unroll
-        for (int j = 0; j < kRB5; ++j) {
-            const int r = r0 + j;
-            const int y = Y0 + r, x = X0 + c;
+        for (int j = 0; j < kRBV; ++j) {
+            const int y = T.Y0 + r0 + j, x = T.X0 + c;
             if (y >= H || x >= W) continue;
-            const float xs = S.x[r + 2 * kLR][c + 2 * kLR], ys = S.y[r + 2 * kLR][c + 2 * kLR];
-            const float dss = fmaf(2.0f * xs, m[1][j], fmaf(ys, m[2][j], m[0][j]));  // n * dS_mean/dI
-            grad[base + (size_t)y * W + x] = fmaf(wl1, (float)S.sgn[r][c], -wss * dss);
+            const float mx = m[0][j], my = m[1][j];  // shifted means
+            const float vxx = fmaf(-mx, mx, m[2][j]), vyy = fmaf(-my, my, m[3][j]);
+            const float vxy = fmaf(-mx, my, m[4][j]);
+            const float ux = mx + sx, uy = my + sy;  // true means
+            const float N1 = fmaf(2.0f * ux, uy, C1), N2 = fmaf(2.0f, vxy, C2);
+            const float D1 = fmaf(ux, ux, fmaf(uy, uy, C1)), D2 = vxx + vyy + C2;
+            const float rD1 = 1.0f / D1, rD2 = 1.0f / D2, rD = rD1 * rD2;
+            const float sv = N1 * N2 * rD;
+            const float dmu = 2.0f * uy * N2 * rD - 2.0f * ux * sv * rD1;
+            const float Bc = -sv * rD2, Cc = 2.0f * N1 * rD;
+            const size_t o = T.base + (size_t)y * W + x;
+            coef[o] = dmu - 2.0f * mx * Bc - my * Cc;  // shifted means: the shift cancels
+            coef[n + o] = Bc;
+            coef[2 * n + o] = Cc;
+            ssum += sv;
         }
     }
 
-    // 6. block partial sums (fixed tree order)
+    // 4. block sums (fixed tree order)
     const int lane = tid & 31, warp = tid >> 5;
 #pragma unroll
     for (int d = 16; d > 0; d >>= 1) {
@@ -264,13 +206,114 @@ __global__ void __launch_bounds__(kLossThreads) k_loss_tile(
     }
     __syncthreads();
     if (tid == 0) {
-        float l = 0.f, s = 0.f;
+        float l = 0.f, sm = 0.f;
         for (int w = 0; w < kLossThreads / 32; ++w) {
             l += S.red[0][w];
-            s += S.red[1][w];
+            sm += S.red[1][w];
         }
         part[2 * (size_t)blockIdx.x] = l;
-        part[2 * (size_t)blockIdx.x + 1] = s;
+        part[2 * (size_t)blockIdx.x + 1] = sm;
+    }
+}
+
+__global__ void __launch_bounds__(kLossThreads) k_loss_grad(
+    const float *__restrict__ img, const float *__restrict__ tgt, int H, int W, int TX, int TY,
+    float lam, double inv_n, const Taps tp_, const float *__restrict__ coef, size_t n,
+    float *__restrict__ grad) {
+    extern __shared__ float4 lsm4[];
+    GradSmem &S = *reinterpret_cast<GradSmem *>(lsm4);
+    const int tid = threadIdx.x;
+    const LossTile T = loss_tile(W, H, TX, TY);
+    const float *ip = img + T.base, *tp = tgt + T.base;
+    const float *g = tp_.t;
+    const size_t mid = (size_t)(H / 2) * W + W / 2;
+    const float sx = ip[mid], sy = tp[mid];
+
+    // 1. stage A, B, Cxy over [Y0 - 5, Y0 + 36] x [X0 - 5, X0 + 36], zero outside the image
+    {
+        float av[3][kLU];
+#pragma unroll
+        for (int u = 0; u < kLU; ++u) {
+            const int i = u * kLossThreads + tid;
+            const int r = i / kLS, c = i - r * kLS;
+            const int y = T.Y0 - kLR + r, x = T.X0 - kLR + c;
+            const bool in = i < kLS * kLS && y >= 0 && y < H && x >= 0 && x < W;
+            const size_t o = in ? T.base + (size_t)y * W + x : 0;
+#pragma unroll
+            for (int q = 0; q < 3; ++q) av[q][u] = in ? coef[q * n + o] : 0.0f;
+        }
+#pragma unroll
+        for (int u = 0; u < kLU; ++u) {
+            const int i = u * kLossThreads + tid;
+            if (i >= kLS * kLS) continue;
+            const int r = i / kLS, c = i - r * kLS;
+#pragma unroll
+            for (int q = 0; q < 3; ++q) S.abc[q][r][c] = av[q][u];
+        }
+    }
+    __syncthreads();
+
+    // 2. horizontal sums of A, B, Cxy
+    for (int it = tid; it < kLS * (kLT / kRBH); it += kLossThreads) {
+        const int r = it / (kLT / kRBH), c0 = (it - r * (kLT / kRBH)) * kRBH;
+        float m[3][kRBH];
+#pragma unroll
+        for (int j = 0; j < kRBH; ++j)
+#pragma unroll
+            for (int q = 0; q < 3; ++q) m[q][j] = 0.0f;
+#pragma unroll
+        for (int k = 0; k < kRBH + kLW - 1; ++k) {
+            float v[3];
+#pragma unroll
+            for (int q = 0; q < 3; ++q) v[q] = S.abc[q][r][c0 + k];
+#pragma unroll
+            for (int j = 0; j < kRBH; ++j) {
+                const int d = k - j;
+                if (d < 0 || d >= kLW) continue;
+#pragma unroll
+                for (int q = 0; q < 3; ++q) m[q][j] = fmaf(g[d], v[q], m[q][j]);
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < 3; ++q)
+#pragma unroll
+            for (int j = 0; j < kRBH; ++j) S.h[q][r][c0 + j] = m[q][j];
+    }
+    __syncthreads();
+
+    // 3. vertical sums -> dL/dI on the tile
+    const float wl1 = (float)((1.0 - (double)lam) * inv_n), wss = (float)((double)lam * inv_n);
+    for (int it = tid; it < (kLT / kRBV) * kLT; it += kLossThreads) {
+        const int rb = it / kLT, c = it - rb * kLT, r0 = rb * kRBV;
+        float m[3][kRBV];
+#pragma unroll
+        for (int j = 0; j < kRBV; ++j)
+#pragma unroll
+            for (int q = 0; q < 3; ++q) m[q][j] = 0.0f;
+#pragma unroll
+        for (int k = 0; k < kRBV + kLW - 1; ++k) {
+            float v[3];
+#pragma unroll
+            for (int q = 0; q < 3; ++q) v[q] = S.h[q][r0 + k][c];
+#pragma unroll
+            for (int j = 0; j < kRBV; ++j) {
+                const int d = k - j;
+                if (d < 0 || d >= kLW) continue;
+#pragma unroll
+                for (int q = 0; q < 3; ++q) m[q][j] = fmaf(g[d], v[q], m[q][j]);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < kRBV; ++j) {
+            const int y = T.Y0 + r0 + j, x = T.X0 + c;
+            if (y >= H || x >= W) continue;
+            const size_t o = (size_t)y * W + x;
+            const float xv = ip[o], yv = tp[o];
+            const float dss = fmaf(2.0f * (xv - sx), m[1][j], fmaf(yv - sy, m[2][j], m[0][j]));
+            const float diff = xv - yv;  // unshifted: ties stay exact zeros
+            const float sg = diff > 0.0f ? 1.0f : (diff < 0.0f ? -1.0f : 0.0f);
+            grad[T.base + o] = fmaf(wl1, sg, -wss * dss);
+        }
     }
 }
 
@@ -319,7 +362,9 @@ size_t pdr_loss_workspace_bytes(int B, int C, int H, int W) {
     int TX, TY;
     long long nb;
     if (!loss_geometry(B, C, H, W, &TX, &TY, &nb)) return 0;
-    return (size_t)(((2 * sizeof(float) * (size_t)nb) + 255) & ~(size_t)255);
+    const size_t part = ((2 * sizeof(float) * (size_t)nb) + 255) & ~(size_t)255;
+    const size_t coef = 3 * sizeof(float) * (size_t)B * C * H * W;  // A, B, Cxy maps
+    return part + ((coef + 255) & ~(size_t)255);
 }
 
 pdr_status pdr_loss_l1_ssim(const float *image, const float *target, int B, int C, int H,
@@ -336,14 +381,18 @@ pdr_status pdr_loss_l1_ssim(const float *image, const float *target, int B, int 
     if ((uintptr_t)workspace & 255) return PDR_ERR_INVALID_ARG;
     if (workspace_bytes < pdr_loss_workspace_bytes(B, C, H, W)) return PDR_ERR_WORKSPACE_TOO_SMALL;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const size_t smem = sizeof(LossSmem);
-    if (cudaFuncSetAttribute(k_loss_tile, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
+    const size_t sc = sizeof(CoefSmem), sg = sizeof(GradSmem);
+    if (cudaFuncSetAttribute(k_loss_coef, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sc) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(k_loss_grad, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sg) !=
+            cudaSuccess)
         return PDR_ERR_CUDA;
-    const double n = (double)B * C * H * W;
+    const size_t n = (size_t)B * C * H * W;
     const float C1 = (0.01f * data_range) * (0.01f * data_range);
     const float C2 = (0.03f * data_range) * (0.03f * data_range);
     float *part = static_cast<float *>(workspace);
+    float *coef = reinterpret_cast<float *>(static_cast<char *>(workspace) +
+                                            (((2 * sizeof(float) * (size_t)nb) + 255) & ~(size_t)255));
     // Window taps exp(-d^2 / (2 sigma^2)), sigma 1.5, normalised to sum 1.
     Taps taps;
     {
@@ -355,10 +404,14 @@ pdr_status pdr_loss_l1_ssim(const float *image, const float *target, int B, int 
         }
         for (int d = 0; d < kLW; ++d) taps.t[d] = (float)(v[d] / sum);
     }
-    k_loss_tile<<<(unsigned)nb, kLossThreads, smem, s>>>(image, target, B * C, H, W, TX, TY, lam,
-                                                         C1, C2, 1.0 / n, taps, grad_image, part);
+    const double inv_n = 1.0 / (double)n;
+    k_loss_coef<<<(unsigned)nb, kLossThreads, sc, s>>>(image, target, H, W, TX, TY, C1, C2, taps,
+                                                       coef, n, part);
     if (cudaGetLastError() != cudaSuccess) return PDR_ERR_CUDA;
-    k_loss_final<<<1, 256, 0, s>>>(part, (int)nb, lam, 1.0 / n, loss);
+    k_loss_grad<<<(unsigned)nb, kLossThreads, sg, s>>>(image, target, H, W, TX, TY, lam, inv_n,
+                                                       taps, coef, n, grad_image);
+    if (cudaGetLastError() != cudaSuccess) return PDR_ERR_CUDA;
+    k_loss_final<<<1, 256, 0, s>>>(part, (int)nb, lam, inv_n, loss);
     return cudaGetLastError() == cudaSuccess ? PDR_OK : PDR_ERR_CUDA;
 }
 
