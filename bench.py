@@ -624,6 +624,37 @@ def run_gpu(args, w):
             sweep[name]["loss_frac"] = lbs.entry(lms, peak_tops)["roofline"]["frac"]
             del lbs
 
+    # A training iteration: render, L1 + SSIM against a target image, backward
+    # from the loss's dL/dI (one graph).
+    train = {}
+    if rank == 0:
+        st = Step(R, torch, w, rank_seed(w, rank), device)
+        tgt = torch.clamp(st.image.new_empty(st.image.shape).normal_(0.5, 0.25), 0, 1)
+        lws = torch.empty(max(R.loss_workspace_bytes(w.B, w.C, w.H, w.W), 256), dtype=torch.uint8,
+                          device=device)
+        lgrad = torch.empty_like(st.image)
+        lval = torch.empty(1, dtype=torch.float32, device=device)
+
+        def train_step():
+            st.fwd()
+            R.l1_ssim_loss(st.image, tgt, 0.2, 1.0, lws, lgrad, lval)
+            R.render_bwd(st.params, lgrad, w.H, w.W, w.k, st.ws, st.dparams, reuse_bins=True)
+
+        st.capture()
+        st._capture("train", [[train_step]])
+        for _ in range(5):
+            flush.fill_(1)
+            st.replay("train")
+        pr = time_graph(st, "train", flush, args.steps, stream)
+        R.check_device_error(st.ws, device)
+        tot = float(pr[:, 0].mean())
+        train = {"ms_per_step": tot, "evals_per_s": st.evals / (tot * 1e-3),
+                 "frames_per_s": w.B / (tot * 1e-3),
+                 "step": "render_fwd (binning inside) + l1_ssim_loss (target ~ clip(N(0.5, 0.25))) "
+                         "+ render_bwd from the loss's dL/dI, one CUDA graph",
+                 "kernels_per_step": graph_kernel_nodes(st.graphs["train"])}
+        del st
+
     # Reduced-precision storage of image and dL/dI (fp32 sums): the same step.
     storage = {}
     if rank == 0:
@@ -694,6 +725,7 @@ def run_gpu(args, w):
             "sweep": sweep,
             "knobs": knobs,
             "storage_half": storage,
+            "train_step": train,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
