@@ -98,6 +98,38 @@ pdr_status check_ws(const Geom &g, void *ws, size_t bytes, Layout *L) {
 
 pdr_status from_cuda(cudaError_t e) { return e == cudaSuccess ? PDR_OK : PDR_ERR_CUDA; }
 
+// Side stream and events of pdr_step_host, one set per host thread and
+// device, created on first use and kept for the thread's lifetime.
+struct StepSide {
+    cudaStream_t side = nullptr;
+    cudaEvent_t ev[4] = {};
+};
+constexpr int kMaxDevices = 64;
+
+cudaError_t step_side(StepSide **out) {
+    static thread_local StepSide sides[kMaxDevices];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    StepSide &d = sides[dev];
+    if (!d.side) {
+        StepSide n;
+        e = cudaStreamCreateWithFlags(&n.side, cudaStreamNonBlocking);
+        for (int j = 0; j < 4 && e == cudaSuccess; ++j)
+            e = cudaEventCreateWithFlags(&n.ev[j], cudaEventDisableTiming);
+        if (e != cudaSuccess) {
+            for (cudaEvent_t v : n.ev)
+                if (v) cudaEventDestroy(v);
+            if (n.side) cudaStreamDestroy(n.side);
+            return e;
+        }
+        d = n;
+    }
+    *out = &d;
+    return cudaSuccess;
+}
+
 cudaError_t bin(const float *params, const Geom &g, const Workspace &ws, cudaStream_t s) {
     return launch_bin(params, g, ws, s);
 }
@@ -255,22 +287,50 @@ pdr_status pdr_step_host(const float *h_params, const float *h_grad_image, float
     st = check_ws(g, workspace, workspace_bytes, &L);
     if (st != PDR_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    StepSide *side = nullptr;
+    st = from_cuda(step_side(&side));
+    if (st != PDR_OK) return st;
+    cudaStream_t s2 = side->side;
+    cudaEvent_t *ev = side->ev;
     const size_t pbytes = sizeof(float) * (size_t)B * N * g.P;
     const size_t ibytes = sizeof(float) * (size_t)B * C * H * W;
-    st = from_cuda(cudaMemcpyAsync(d_params, h_params, pbytes, cudaMemcpyHostToDevice, s));
-    if (st != PDR_OK) return st;
-    st = from_cuda(cudaMemcpyAsync(d_grad_image, h_grad_image, ibytes, cudaMemcpyHostToDevice, s));
-    if (st != PDR_OK) return st;
+    // stream:  params H2D | forward (bins inside) | .. backward | grads D2H | join
+    // side:                 | dL/dI H2D ..         | image D2H ..
+    // The side stream starts after everything already on `stream` (ev[0]), so a
+    // previous step's backward is done with d_grad_image before it is
+    // overwritten, and `stream` joins the side stream at the end (ev[3]).
+    const cudaError_t e = [&]() -> cudaError_t {
+        cudaError_t r;
+        if ((r = cudaMemcpyAsync(d_params, h_params, pbytes, cudaMemcpyHostToDevice, s))) return r;
+        if ((r = cudaEventRecord(ev[0], s))) return r;
+        if ((r = cudaStreamWaitEvent(s2, ev[0], 0))) return r;
+        if ((r = cudaMemcpyAsync(d_grad_image, h_grad_image, ibytes, cudaMemcpyHostToDevice, s2)))
+            return r;
+        return cudaEventRecord(ev[1], s2);
+    }();
+    if (e != cudaSuccess) return PDR_ERR_CUDA;
     st = pdr_render_fwd(d_params, B, N, C, H, W, k, d_image, workspace, workspace_bytes, 0,
                         stream);
-    if (st != PDR_OK) return st;
+    if (st != PDR_OK) {  // still join the side stream, so that `stream` covers its copy
+        if (cudaEventRecord(ev[3], s2) == cudaSuccess) cudaStreamWaitEvent(s, ev[3], 0);
+        return st;
+    }
+    const cudaError_t e2 = [&]() -> cudaError_t {
+        cudaError_t r;
+        if ((r = cudaEventRecord(ev[2], s))) return r;
+        if ((r = cudaStreamWaitEvent(s2, ev[2], 0))) return r;
+        if ((r = cudaMemcpyAsync(h_image, d_image, ibytes, cudaMemcpyDeviceToHost, s2))) return r;
+        if ((r = cudaEventRecord(ev[3], s2))) return r;
+        return cudaStreamWaitEvent(s, ev[1], 0);
+    }();
+    if (e2 != cudaSuccess) return PDR_ERR_CUDA;
     st = pdr_render_bwd(d_params, d_grad_image, B, N, C, H, W, k, d_grad_params, workspace,
                         workspace_bytes, 1, stream);
     if (st != PDR_OK) return st;
-    st = from_cuda(cudaMemcpyAsync(h_image, d_image, ibytes, cudaMemcpyDeviceToHost, s));
+    st = from_cuda(cudaMemcpyAsync(h_grad_params, d_grad_params, pbytes,
+                                   cudaMemcpyDeviceToHost, s));
     if (st != PDR_OK) return st;
-    return from_cuda(cudaMemcpyAsync(h_grad_params, d_grad_params, pbytes,
-                                     cudaMemcpyDeviceToHost, s));
+    return from_cuda(cudaStreamWaitEvent(s, ev[3], 0));
 }
 
 pdr_status pdr_check_device_error(void *workspace, void *stream) {

@@ -137,9 +137,14 @@ long long pdr_list_capacity_per_frame(int N, int k);
  * copies h_params and h_grad_image to the caller's device buffers d_params and
  * d_grad_image, renders forward into d_image, runs the backward into
  * d_grad_params, and copies the image and the gradients back to h_image and
- * h_grad_params -- all enqueued on `stream` (one cudaMemcpyAsync per buffer;
- * pinned host memory makes the copies asynchronous).  The call returns after
- * enqueueing; synchronise the stream before reading h_image / h_grad_params. */
+ * h_grad_params (one cudaMemcpyAsync per buffer; pinned host memory makes
+ * the copies asynchronous).  The params copy, the forward, the backward and
+ * the gradient copy run on `stream`; the dL/dI copy (overlapping the forward)
+ * and the image copy-back (overlapping the backward) run on a side stream of
+ * the library (one per host thread and device, created on first use), which
+ * starts after the work already on `stream` and which `stream` joins before
+ * the call's last operation.  The call returns after enqueueing; synchronise
+ * `stream` before reading h_image / h_grad_params. */
 pdr_status pdr_step_host(const float *h_params, const float *h_grad_image,
                          float *h_image, float *h_grad_params, int B, int N,
                          int C, int H, int W, int k, float *d_params,

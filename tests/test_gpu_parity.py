@@ -198,6 +198,33 @@ def test_host_step_matches_device_path():
     assert np.array_equal(h_dp.numpy(), dp)
 
 
+def test_host_steps_back_to_back_on_one_stream():
+    """Consecutive host steps share the device buffers; only the caller's
+    stream is synchronised, so the library's side-stream copies must be
+    ordered after the previous step and joined back into that stream."""
+    w = WORKLOADS["mono64"].scaled(B=4)
+    pa, ga = make_inputs(w)
+    pb, gb = make_inputs(w.scaled(seed=w.seed + 1))
+    ref_a = run_gpu(pa, ga, w.H, w.W, w.k)
+    ref_b = run_gpu(pb, gb, w.H, w.W, w.k)
+    hosts = [(torch.from_numpy(p).pin_memory(), torch.from_numpy(g).pin_memory())
+             for p, g in ((pa, ga), (pb, gb))]
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        _, _, bufs = R.step_host(*hosts[0], w.H, w.W, w.k)
+        outs = []
+        for j in (1, 0, 1):
+            mine = dict(bufs)
+            mine["h_image"] = torch.empty_like(bufs["h_image"]).pin_memory()
+            mine["h_grad_params"] = torch.empty_like(bufs["h_grad_params"]).pin_memory()
+            outs.append((j,) + R.step_host(*hosts[j], w.H, w.W, w.k, mine)[:2])
+        stream.synchronize()
+    for j, h_img, h_dp in outs:
+        img, dp = (ref_a, ref_b)[j]
+        assert np.array_equal(h_img.numpy(), img)
+        assert np.array_equal(h_dp.numpy(), dp)
+
+
 def test_invalid_arguments_rejected_on_device_buffers():
     p = torch.zeros((1, 4, 6), device="cuda")
     with pytest.raises(ValueError):
