@@ -328,12 +328,16 @@ size_t bin_scatter_smem(const Geom &g) {
     return sizeof(int) * (size_t)g.T * (g.scatter_warps + 2);
 }
 
+// Dynamic shared memory above which a launch needs the opt-in attribute: the
+// 48 KB default less room for the kernel's static arrays.
+constexpr size_t kStaticSmemRoom = 44 * 1024;
+
 cudaError_t launch_bin(const float *params, const Geom &g, const Workspace &ws,
                        cudaStream_t s) {
     cudaError_t e;
     if (g.frame_block) {
         const size_t sf = bin_frame_smem(g);
-        if (sf > 48 * 1024) {
+        if (sf > kStaticSmemRoom) {
             e = cudaFuncSetAttribute(k_bin_frame, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)sf);
             if (e != cudaSuccess) return e;

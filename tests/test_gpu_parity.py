@@ -262,6 +262,22 @@ def test_chunked_binning_paths(B, N, C, H, W, k):
     check_all(p, g, H, W, k)
 
 
+@pytest.mark.parametrize("B,N,C,H,W,k", [
+    (3, 1000, 2, 96, 160, 11),   # 60 tiles
+    (2, 4000, 1, 128, 128, 9),   # 64 tiles, 4000 ids
+    (5, 333, 4, 32, 64, 9),      # 8 tiles, a ragged last warp of ids
+    (2, 5000, 3, 48, 80, 7),     # 15 tiles, 5000 ids
+    (1, 980, 1, 192, 256, 5),    # 192 tiles x 31 warps: tables of exactly 48 KB + static arrays
+])
+def test_frame_block_binning(B, N, C, H, W, k):
+    """Frames binned by one block each (up to 256 tiles), windows partly and
+    wholly off the grid, ragged last warp of ids."""
+    rng = np.random.default_rng(B * 7 + N + W)
+    p = _edge_params(rng, B, N, C, H, W, k)
+    g = rng.standard_normal((B, C, H, W)).astype(np.float32)
+    check_all(p, g, H, W, k)
+
+
 @pytest.mark.parametrize("B", [149, 300, 450])
 def test_many_small_frames(B):
     """More frames than SMs: smaller frame-binning blocks, one wave."""
