@@ -225,6 +225,40 @@ def test_host_steps_back_to_back_on_one_stream():
         assert np.array_equal(h_dp.numpy(), dp)
 
 
+def test_host_steps_from_two_threads():
+    """Two host threads, each with its own stream and buffers, run host steps
+    at the same time; each thread's side stream and events are its own."""
+    import threading
+    w = WORKLOADS["mono64"].scaled(B=3)
+    inputs = [make_inputs(w.scaled(seed=w.seed + j)) for j in range(2)]
+    refs = [run_gpu(p, g, w.H, w.W, w.k) for p, g in inputs]
+    results, errors = [None, None], []
+
+    def worker(j):
+        try:
+            hp = torch.from_numpy(inputs[j][0]).pin_memory()
+            hg = torch.from_numpy(inputs[j][1]).pin_memory()
+            stream = torch.cuda.Stream()
+            with torch.cuda.stream(stream):
+                bufs = None
+                for _ in range(5):
+                    h_img, h_dp, bufs = R.step_host(hp, hg, w.H, w.W, w.k, bufs)
+                stream.synchronize()
+            results[j] = (h_img.numpy().copy(), h_dp.numpy().copy())
+        except Exception as e:  # reported below, in the main thread
+            errors.append(e)
+
+    threads = [threading.Thread(target=worker, args=(j,)) for j in range(2)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    assert not errors, errors
+    for j in range(2):
+        assert np.array_equal(results[j][0], refs[j][0])
+        assert np.array_equal(results[j][1], refs[j][1])
+
+
 def test_invalid_arguments_rejected_on_device_buffers():
     p = torch.zeros((1, 4, 6), device="cuda")
     with pytest.raises(ValueError):
