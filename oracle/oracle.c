@@ -36,7 +36,9 @@
  *   - a Gaussian with non-finite mu, or whose window misses the grid,
  *     contributes nothing and gets zero gradients;
  *   - the binning reference assigns Gaussian i to every 16 x 16 tile its
- *     clipped window touches, tiles in row-major order, ids ascending.
+ *     clipped window touches, tiles in row-major order, ids ascending;
+ *   - a frame may hold no Gaussians (N = 0): the empty sum, an all-zero
+ *     image, no gradients and empty tile lists.
  *
  * Layouts: params [B][N][5+C] (mu_x, mu_y, s_1, s_2, theta, a_0..), fp32 for
  * the *_fwd / *_bwd / bin entry points and fp64 for the *_f64 ones (used by the
@@ -55,8 +57,9 @@
 
 #define TILE 16
 
+/* N = 0 is a frame with no Gaussians: the empty sum renders to zero. */
 static int bad_sizes(int B, int N, int C, int H, int W, int k) {
-    return B < 1 || N < 1 || C < 1 || H < 1 || W < 1 || k < 1 || (k % 2) == 0;
+    return B < 1 || N < 0 || C < 1 || H < 1 || W < 1 || k < 1 || (k % 2) == 0;
 }
 
 /* Clipped window of one Gaussian along one axis: pixels [lo, hi] of [0, n).
@@ -85,7 +88,7 @@ int oracle_max_threads(void) {
 /* Forward render: image[b][c][y][x] = sum_i a_ic w_i(x, y), i ascending. */
 int oracle_render_fwd_f64(const double *params, int B, int N, int C, int H,
                           int W, int k, double *image, int nthreads) {
-    if (bad_sizes(B, N, C, H, W, k) || !params || !image) return -1;
+    if (bad_sizes(B, N, C, H, W, k) || (N > 0 && !params) || !image) return -1;
     const int P = 5 + C;
     const int r = (k - 1) / 2;
     if (nthreads < 1) nthreads = 1;
@@ -129,7 +132,7 @@ int oracle_render_fwd_f64(const double *params, int B, int N, int C, int H,
 int oracle_render_bwd_f64(const double *params, const double *grad_image,
                           int B, int N, int C, int H, int W, int k,
                           double *grad_params, int nthreads) {
-    if (bad_sizes(B, N, C, H, W, k) || !params || !grad_image || !grad_params)
+    if (bad_sizes(B, N, C, H, W, k) || (N > 0 && (!params || !grad_params)) || !grad_image)
         return -1;
     const int P = 5 + C;
     const int r = (k - 1) / 2;
@@ -191,7 +194,7 @@ static double *widen(const float *src, size_t n) {
 
 int oracle_render_fwd(const float *params, int B, int N, int C, int H, int W,
                       int k, double *image, int nthreads) {
-    if (bad_sizes(B, N, C, H, W, k) || !params || !image) return -1;
+    if (bad_sizes(B, N, C, H, W, k) || (N > 0 && !params) || !image) return -1;
     double *p = widen(params, (size_t)B * N * (5 + C));
     if (!p) return -2;
     int rc = oracle_render_fwd_f64(p, B, N, C, H, W, k, image, nthreads);
@@ -202,7 +205,7 @@ int oracle_render_fwd(const float *params, int B, int N, int C, int H, int W,
 int oracle_render_bwd(const float *params, const float *grad_image, int B, int N,
                       int C, int H, int W, int k, double *grad_params,
                       int nthreads) {
-    if (bad_sizes(B, N, C, H, W, k) || !params || !grad_image || !grad_params)
+    if (bad_sizes(B, N, C, H, W, k) || (N > 0 && (!params || !grad_params)) || !grad_image)
         return -1;
     double *p = widen(params, (size_t)B * N * (5 + C));
     double *g = widen(grad_image, (size_t)B * C * H * W);
@@ -222,7 +225,7 @@ int oracle_render_bwd(const float *params, const float *grad_image, int B, int N
  * they fit in cap (pass tile_ids = NULL, cap = 0 to count). */
 long long oracle_bin(const float *params, int B, int N, int C, int H, int W, int k,
                      long long *tile_offsets, int *tile_ids, long long cap) {
-    if (bad_sizes(B, N, C, H, W, k) || !params) return -1;
+    if (bad_sizes(B, N, C, H, W, k) || (N > 0 && !params)) return -1;
     const int P = 5 + C;
     const int r = (k - 1) / 2;
     const int TX = (W + TILE - 1) / TILE, TY = (H + TILE - 1) / TILE;

@@ -233,6 +233,20 @@ def test_additivity_over_gaussian_sets():
     assert np.abs(both - parts).max() <= 1e-13 * np.abs(both).max()
 
 
+def test_a_frame_without_gaussians():
+    """N = 0, the empty sum: an all-zero image, no gradients, empty tile lists;
+    and splitting a set into itself and the empty set changes nothing."""
+    p, H, W = _random_params(4)
+    empty = p[:, :0]
+    img = oracle.render_fwd(empty, H, W, 9)
+    assert img.shape == (p.shape[0], p.shape[2] - 5, H, W) and not img.any()
+    g = np.random.default_rng(9).standard_normal(img.shape).astype(np.float32)
+    assert oracle.render_bwd(empty, g, H, W, 9).shape == (p.shape[0], 0, p.shape[2])
+    offs, ids = oracle.bin_tiles(empty, H, W, 9)
+    assert not offs.any() and ids.size == 0
+    assert np.array_equal(oracle.render_fwd(p, H, W, 9), oracle.render_fwd(p, H, W, 9) + img)
+
+
 def test_isotropic_theta_invariance_and_zero_theta_grad():
     p, H, W = _random_params(5)
     p[..., 3] = p[..., 2]
