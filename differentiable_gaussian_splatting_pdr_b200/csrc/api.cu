@@ -24,7 +24,8 @@ struct Layout {
 };
 
 pdr_status make_geom(int B, int N, int C, int H, int W, int k, Geom *g) {
-    if (B < 1 || N < 1 || C < 1 || H < 1 || W < 1 || k < 1 || (k & 1) == 0)
+    // N = 0: frames with no Gaussians (the entry points launch no kernel then).
+    if (B < 1 || N < 0 || C < 1 || H < 1 || W < 1 || k < 1 || (k & 1) == 0)
         return PDR_ERR_INVALID_ARG;
     if (C > PDR_MAX_C || k > PDR_MAX_K) return PDR_ERR_TOO_LARGE;
     const long long TX = (W + kTile - 1) / kTile, TY = (H + kTile - 1) / kTile;
@@ -50,6 +51,7 @@ pdr_status make_geom(int B, int N, int C, int H, int W, int k, Geom *g) {
     g->frame_block = T <= kFrameBlockMaxT && N <= kFrameBlockMaxN;
     int ft = ((N + 31) / 32) * 32;
     if (ft > 1024) ft = 1024;
+    if (ft < 32) ft = 32;
     // More frames than SMs: smaller blocks, so that all frames are resident in
     // one wave (about 1024 binning threads per SM).
     const long long per_sm = ((long long)B + 147) / 148;
@@ -131,8 +133,16 @@ cudaError_t step_side(StepSide **out) {
 }
 
 cudaError_t bin(const float *params, const Geom &g, const Workspace &ws, cudaStream_t s) {
+    if (g.N == 0) {  // no Gaussians: a clear error word and every tile list empty at 0
+        cudaError_t e = cudaMemsetAsync(ws.err, 0, sizeof(int), s);
+        if (e != cudaSuccess) return e;
+        return cudaMemsetAsync(ws.offs, 0, sizeof(int) * (size_t)g.B * (g.T + 1), s);
+    }
     return launch_bin(params, g, ws, s);
 }
+
+// params (and grad_params) may be null only when there are no Gaussians.
+bool params_ok(const Geom &g, const void *p) { return g.N == 0 || p != nullptr; }
 
 bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3) == 0; }
 
@@ -175,7 +185,7 @@ pdr_status pdr_build_bins(const float *params, int B, int N, int C, int H, int W
     Geom g;
     pdr_status st = make_geom(B, N, C, H, W, k, &g);
     if (st != PDR_OK) return st;
-    if (!params || !aligned4(params)) return PDR_ERR_INVALID_ARG;
+    if (!params_ok(g, params) || !aligned4(params)) return PDR_ERR_INVALID_ARG;
     Layout L;
     st = check_ws(g, workspace, workspace_bytes, &L);
     if (st != PDR_OK) return st;
@@ -194,13 +204,20 @@ pdr_status pdr_render_fwd_ex(const float *params, int B, int N, int C, int H, in
     Geom g;
     pdr_status st = make_geom(B, N, C, H, W, k, &g);
     if (st != PDR_OK) return st;
-    if (!params || !image || !aligned4(params) || !dtype_ok(image_dtype, image))
+    if (!params_ok(g, params) || !image || !aligned4(params) || !dtype_ok(image_dtype, image))
         return PDR_ERR_INVALID_ARG;
     Layout L;
     st = check_ws(g, workspace, workspace_bytes, &L);
     if (st != PDR_OK) return st;
     const Workspace ws = carve(workspace, L);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (g.N == 0) {  // the empty sum (all-zero bits are 0.0 in every storage type)
+        st = from_cuda(bin(params, g, ws, s));
+        if (st != PDR_OK) return st;
+        const size_t esize = image_dtype == PDR_F32 ? sizeof(float) : 2;
+        return from_cuda(
+            cudaMemsetAsync(image, 0, esize * (size_t)g.B * g.C * g.H * g.W, s));
+    }
     g.img_dtype = image_dtype;
     g.out_vec2 = ((g.W & 1) == 0) && ((reinterpret_cast<uintptr_t>(image) & 7) == 0);
     g.out_vec4 = ((g.W & 3) == 0) && ((reinterpret_cast<uintptr_t>(image) & 15) == 0);
@@ -227,12 +244,13 @@ pdr_status pdr_render_bwd_ex(const float *params, const void *grad_image, int gr
     Geom g;
     pdr_status st = make_geom(B, N, C, H, W, k, &g);
     if (st != PDR_OK) return st;
-    if (!params || !grad_image || !grad_params || !aligned4(params) ||
-        !dtype_ok(grad_dtype, grad_image) || !aligned4(grad_params))
+    if (!params_ok(g, params) || !grad_image || !params_ok(g, grad_params) ||
+        !aligned4(params) || !dtype_ok(grad_dtype, grad_image) || !aligned4(grad_params))
         return PDR_ERR_INVALID_ARG;
     Layout L;
     st = check_ws(g, workspace, workspace_bytes, &L);
     if (st != PDR_OK) return st;
+    if (g.N == 0) return PDR_OK;  // no Gaussians: no gradients to write
     const Workspace ws = carve(workspace, L);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     g.img_dtype = grad_dtype;
@@ -257,7 +275,8 @@ pdr_status pdr_bin(const float *params, int B, int N, int C, int H, int W, int k
     Geom g;
     pdr_status st = make_geom(B, N, C, H, W, k, &g);
     if (st != PDR_OK) return st;
-    if (!params || !tile_offsets || !tile_ids || !aligned4(params)) return PDR_ERR_INVALID_ARG;
+    if (!params_ok(g, params) || !tile_offsets || (g.N > 0 && !tile_ids) || !aligned4(params))
+        return PDR_ERR_INVALID_ARG;
     Layout L;
     st = check_ws(g, workspace, workspace_bytes, &L);
     if (st != PDR_OK) return st;
@@ -267,7 +286,7 @@ pdr_status pdr_bin(const float *params, int B, int N, int C, int H, int W, int k
     if (st != PDR_OK) return st;
     st = from_cuda(cudaMemcpyAsync(tile_offsets, ws.offs, sizeof(int) * (size_t)g.B * (g.T + 1),
                                    cudaMemcpyDeviceToDevice, s));
-    if (st != PDR_OK) return st;
+    if (st != PDR_OK || g.cap == 0) return st;
     return from_cuda(cudaMemcpyAsync(tile_ids, ws.ids, sizeof(int) * (size_t)g.B * g.cap,
                                      cudaMemcpyDeviceToDevice, s));
 }
@@ -280,8 +299,8 @@ pdr_status pdr_step_host(const float *h_params, const float *h_grad_image, float
     Geom g;
     pdr_status st = make_geom(B, N, C, H, W, k, &g);
     if (st != PDR_OK) return st;
-    if (!h_params || !h_grad_image || !h_image || !h_grad_params || !d_params ||
-        !d_grad_image || !d_image || !d_grad_params)
+    if (!params_ok(g, h_params) || !h_grad_image || !h_image || !params_ok(g, h_grad_params) ||
+        !params_ok(g, d_params) || !d_grad_image || !d_image || !params_ok(g, d_grad_params))
         return PDR_ERR_INVALID_ARG;
     Layout L;
     st = check_ws(g, workspace, workspace_bytes, &L);
@@ -301,7 +320,8 @@ pdr_status pdr_step_host(const float *h_params, const float *h_grad_image, float
     // overwritten, and `stream` joins the side stream at the end (ev[3]).
     const cudaError_t e = [&]() -> cudaError_t {
         cudaError_t r;
-        if ((r = cudaMemcpyAsync(d_params, h_params, pbytes, cudaMemcpyHostToDevice, s))) return r;
+        if (pbytes && (r = cudaMemcpyAsync(d_params, h_params, pbytes, cudaMemcpyHostToDevice, s)))
+            return r;
         if ((r = cudaEventRecord(ev[0], s))) return r;
         if ((r = cudaStreamWaitEvent(s2, ev[0], 0))) return r;
         if ((r = cudaMemcpyAsync(d_grad_image, h_grad_image, ibytes, cudaMemcpyHostToDevice, s2)))
@@ -327,9 +347,11 @@ pdr_status pdr_step_host(const float *h_params, const float *h_grad_image, float
     st = pdr_render_bwd(d_params, d_grad_image, B, N, C, H, W, k, d_grad_params, workspace,
                         workspace_bytes, 1, stream);
     if (st != PDR_OK) return st;
-    st = from_cuda(cudaMemcpyAsync(h_grad_params, d_grad_params, pbytes,
-                                   cudaMemcpyDeviceToHost, s));
-    if (st != PDR_OK) return st;
+    if (pbytes) {
+        st = from_cuda(cudaMemcpyAsync(h_grad_params, d_grad_params, pbytes,
+                                       cudaMemcpyDeviceToHost, s));
+        if (st != PDR_OK) return st;
+    }
     return from_cuda(cudaStreamWaitEvent(s, ev[3], 0));
 }
 

@@ -47,8 +47,8 @@ cudaError_t scratch_address(void **out) {
 
 extern "C" pdr_status pdr_render_fwd_noalloc(const float *params, int B, int N, int C, int H,
                                              int W, int k, float *image, void *stream) {
-    if (B < 1 || N < 1 || C < 1 || H < 1 || W < 1 || k < 1 || (k & 1) == 0 || !params ||
-        !image)
+    if (B < 1 || N < 0 || C < 1 || H < 1 || W < 1 || k < 1 || (k & 1) == 0 ||
+        (N > 0 && !params) || !image)
         return PDR_ERR_INVALID_ARG;
     const size_t need = pdr_workspace_bytes(B, N, C, H, W, k);
     if (need == 0 || need > PDR_STATIC_SCRATCH_BYTES) return PDR_ERR_TOO_LARGE;

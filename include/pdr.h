@@ -33,10 +33,15 @@
  * up at the caller's next synchronisation.
  *
  * Validation (host side, before anything is launched; on failure nothing is
- * launched and outputs are untouched): B, N, C, H, W >= 1; k odd and >= 1;
- * sizes within the limits below (else PDR_ERR_TOO_LARGE); non-null pointers;
- * workspace_bytes >= pdr_workspace_bytes(...) and a 256-byte aligned
- * workspace.
+ * launched and outputs are untouched): B, C, H, W >= 1 and N >= 0; k odd and
+ * >= 1; sizes within the limits below (else PDR_ERR_TOO_LARGE); non-null
+ * pointers, except that the arrays sized by N (params, grad_params, tile_ids)
+ * may be NULL when N = 0; workspace_bytes >= pdr_workspace_bytes(...) and a
+ * 256-byte aligned workspace.
+ *
+ * Frames with no Gaussians (N = 0) are the empty sum: the forward zeroes the
+ * image and leaves empty bins, the backward writes nothing, pdr_bin writes
+ * all-zero offsets; no kernel is launched (stream-ordered memsets only).
  *
  * Numerics: fp32 arithmetic with a hardware base-2 exponential; fixed
  * summation order (every list is in ascending Gaussian id), so results are

@@ -52,7 +52,7 @@ def test_status_strings(lib):
 
 
 @pytest.mark.parametrize("args", [
-    (0, 10, 1, 32, 32, 7), (1, 0, 1, 32, 32, 7), (1, 10, 0, 32, 32, 7),
+    (0, 10, 1, 32, 32, 7), (1, -1, 1, 32, 32, 7), (1, 10, 0, 32, 32, 7),
     (1, 10, 1, 0, 32, 7), (1, 10, 1, 32, 0, 7), (1, 10, 1, 32, 32, 0),
     (1, 10, 1, 32, 32, 8), (1, 10, 1, 32, 32, -3),
     (1, 10, 9, 32, 32, 7),            # C beyond PDR_MAX_C
@@ -61,6 +61,14 @@ def test_status_strings(lib):
 ])
 def test_workspace_bytes_rejects_bad_sizes(lib, args):
     assert lib.pdr_workspace_bytes(*args) == 0
+
+
+def test_frames_without_gaussians_are_valid_sizes(lib):
+    """N = 0 (the empty sum) is accepted: a workspace for the bins' offsets, no
+    list capacity."""
+    n0 = lib.pdr_workspace_bytes(3, 0, 2, 40, 24, 9)
+    assert 0 < n0 < lib.pdr_workspace_bytes(3, 1, 2, 40, 24, 9)
+    assert lib.pdr_list_capacity_per_frame(0, 9) == 0
 
 
 def _max_tiles_touched(k):
@@ -119,6 +127,20 @@ def test_bwd_bin_and_host_step_validation(lib):
     assert lib.pdr_step_host(FAKE, FAKE, FAKE, None, 2, 64, 3, 40, 24, 9,
                              FAKE, FAKE, FAKE, FAKE, FAKE, ws, None) == 1
     assert lib.pdr_check_device_error(None, None) == 1
+
+
+@no_gpu
+def test_null_arrays_only_for_frames_without_gaussians(lib):
+    """params / grad_params / tile_ids may be NULL only when N = 0; the N = 0
+    calls here stop at the workspace check (size 16), before any launch."""
+    ws = lib.pdr_workspace_bytes(2, 64, 3, 40, 24, 9)
+    assert lib.pdr_render_fwd(None, 2, 64, 3, 40, 24, 9, FAKE, FAKE, ws, 0, None) == 1
+    assert lib.pdr_render_fwd(None, 2, 0, 3, 40, 24, 9, FAKE, FAKE, 16, 0, None) == 2
+    assert lib.pdr_render_bwd(None, FAKE, 2, 0, 3, 40, 24, 9, None, FAKE, 16, 1, None) == 2
+    assert lib.pdr_render_bwd(None, None, 2, 0, 3, 40, 24, 9, None, FAKE, 16, 1, None) == 1
+    assert lib.pdr_bin(None, 2, 0, 3, 40, 24, 9, FAKE, None, FAKE, 16, None) == 2
+    assert lib.pdr_bin(None, 2, 64, 3, 40, 24, 9, FAKE, None, FAKE, ws, None) == 1
+    assert lib.pdr_render_fwd(None, 2, -1, 3, 40, 24, 9, FAKE, FAKE, ws, 0, None) == 1
 
 
 def test_binding_fails_loudly_without_library(tmp_path):

@@ -259,6 +259,33 @@ def test_host_steps_from_two_threads():
         assert np.array_equal(results[j][1], refs[j][1])
 
 
+@pytest.mark.parametrize("B,C,H,W,k", [(2, 3, 40, 24, 9), (3, 1, 64, 64, 9), (1, 4, 128, 96, 15)])
+def test_frames_without_gaussians(B, C, H, W, k):
+    """N = 0, the empty sum: zero images (every storage type, overwriting what
+    was there), no gradients, all-zero tile offsets, also through the host
+    step and autograd."""
+    rng = np.random.default_rng(B + H)
+    p = np.zeros((B, 0, 5 + C), dtype=np.float32)
+    g = rng.standard_normal((B, C, H, W)).astype(np.float32)
+    check_bins(p, H, W, k)
+    pt, gt = torch.from_numpy(p).cuda(), torch.from_numpy(g).cuda()
+    for dtype in (torch.float32, torch.float16, torch.bfloat16):
+        out = torch.full((B, C, H, W), 7.0, dtype=dtype, device="cuda")
+        img, ws = R.render_fwd(pt, H, W, k, out=out, dtype=dtype)
+        dp = R.render_bwd(pt, gt, H, W, k, ws)
+        R.check_device_error(ws)
+        assert not img.any() and dp.shape == (B, 0, 5 + C)
+    offs, ids, cap = R.bin_tiles(pt, H, W, k)
+    assert cap == 0 and ids.numel() == 0 and not offs.any()
+    h_img, h_dp, _ = R.step_host(torch.from_numpy(p).pin_memory(),
+                                 torch.from_numpy(g).pin_memory(), H, W, k)
+    torch.cuda.synchronize()
+    assert not h_img.any() and h_dp.shape == (B, 0, 5 + C)
+    pa = pt.clone().requires_grad_(True)
+    (R.render(pa, H, W, k) * gt).sum().backward()
+    assert pa.grad is not None and pa.grad.shape == pa.shape
+
+
 def test_invalid_arguments_rejected_on_device_buffers():
     p = torch.zeros((1, 4, 6), device="cuda")
     with pytest.raises(ValueError):

@@ -79,3 +79,10 @@ def test_noalloc_rejects_sizes_beyond_its_scratch(lib):
     st = lib.pdr_render_fwd_noalloc(p.data_ptr(), w.B, w.N, w.C, w.H, w.W, w.k,
                                     img.data_ptr(), _stream())
     assert st == PDR_ERR_TOO_LARGE
+
+
+def test_noalloc_frame_without_gaussians(lib):
+    """N = 0: the image is zeroed (the empty sum), params may be NULL."""
+    p = torch.zeros((2, 0, 7), device="cuda")
+    got = _noalloc(lib, p, 40, 24, 9)
+    assert got.shape == (2, 2, 40, 24) and not got.any()
