@@ -140,6 +140,7 @@ def _edge_params(rng, B, N, C, H, W, k, smean=0.4, ssd=0.4):
     (1, 250, 1, 37, 29, 15),
     (3, 80, 3, 16, 16, 3),
     (2, 120, 4, 30, 45, 7),
+    (1, 64, 8, 40, 40, 31),     # largest C with the largest window: the biggest backward halo
 ])
 def test_edge_shapes(B, N, C, H, W, k):
     rng = np.random.default_rng(B * 1000 + N + C)
@@ -314,6 +315,7 @@ def test_separate_bins_then_render_matches_one_call():
 @pytest.mark.parametrize("B,N,C,H,W,k", [
     (2, 40000, 1, 112, 144, 5),   # large frames: chunked count, two scan passes, 63 tiles
     (1, 20000, 2, 300, 240, 3),   # 285 tiles (more than one frame block takes), 20 chunks
+    (1, 3000, 1, 2048, 2048, 5),  # the most tiles a frame may have (16384): 1-warp scatter blocks
 ])
 def test_chunked_binning_paths(B, N, C, H, W, k):
     """Frames too large for one binning block (count, two-level scan, scatter)."""
