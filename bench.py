@@ -193,16 +193,17 @@ class ClockSampler:
 # ----------------------------------------------------------------------------
 # the oracle (CPU baseline and reference arm)
 # ----------------------------------------------------------------------------
-def oracle_sample(w, seconds: float, max_frames=None):
-    """Time the fp64 oracle fwd + bwd on the host cores over a bounded sample
-    of workload w: whole batches (or the first max_frames frames) repeated
-    until `seconds` have passed.  Returns (evals/s, frames/s, cores, sample)."""
+def oracle_sample(w, seconds: float, max_frames=None, threads=None):
+    """Time the fp64 oracle fwd + bwd on the host cores (all of them, or
+    `threads`) over a bounded sample of workload w: whole batches (or the first
+    max_frames frames) repeated until `seconds` have passed.  Returns
+    (evals/s, frames/s, cores, sample, seconds per repetition)."""
     import oracle  # test infrastructure: only the CPU-baseline leg runs it
     B = w.B if max_frames is None else min(w.B, max_frames)
     p, g = make_inputs(w)
     p, g = p[:B].copy(), g[:B].copy()
     ev = in_grid_evals(p, w.H, w.W, w.k)
-    cores = oracle.max_threads()
+    cores = oracle.max_threads() if threads is None else max(1, int(threads))
     reps, t0 = 0, time.perf_counter()
     while True:
         oracle.render_fwd(p, w.H, w.W, w.k, cores)
@@ -693,6 +694,9 @@ def run_gpu(args, w):
         v, fps, cores, sample, _ = oracle_sample(w, args.cpu_seconds)
         cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
                "frames_per_s": fps}
+        v1, fps1, _, sample1, _ = oracle_sample(w, min(3.0, args.cpu_seconds), threads=1)
+        cpu["single_core"] = {"value": v1, "unit": UNIT, "cores": 1, "sample": sample1,
+                              "frames_per_s": fps1}
 
     if rank == 0:
         launches_per_step = graph_kernel_nodes(step.graphs["main"])

@@ -106,3 +106,13 @@ def test_reference_arm_under_torchrun_two_ranks():
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["steps"] == 2
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
     assert d["value"] > 0 and d["cpu_baseline"]["value"] == d["value"]
+
+
+def test_oracle_sample_on_one_core_and_on_all():
+    """The CPU baseline's two figures: the oracle on every host core and on one."""
+    w = WORKLOADS["tiny"]
+    v1, f1, c1, s1, _ = bench.oracle_sample(w, 0.05, threads=1)
+    va, fa, ca, sa, _ = bench.oracle_sample(w, 0.05)
+    assert c1 == 1 and ca >= 1
+    assert v1 > 0 and va > 0 and f1 > 0 and fa > 0
+    assert "frames of tiny" in s1 and "frames of tiny" in sa
