@@ -2,7 +2,7 @@
 // clipped k x k window touches, lists in ascending Gaussian id so that every
 // fp32 sum downstream has a fixed order.  The additive accumulation (reading
 // notes, "Method") has no depth order, so any fixed order is correct;
-// ascending id is the one the oracle also uses.  Three kernels on the
+// ascending id is the one the oracle also uses.  Four kernels on the
 // caller's stream, no float atomics, no host synchronisation:
 //
 //   k_count   one block per (frame, chunk of kBinChunk Gaussians): the
