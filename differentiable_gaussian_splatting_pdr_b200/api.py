@@ -174,9 +174,11 @@ def step_host(h_params: torch.Tensor, h_grad_image: torch.Tensor, H: int, W: int
     """One forward + backward pass from host (ideally pinned) tensors.
 
     Copies inputs to the device, renders, back-propagates dL/dI, and copies the
-    image and dL/dparams back, all enqueued on the current stream by one C-ABI
-    call (pdr_step_host).  Returns (h_image, h_grad_params, dev_bufs); the
-    host outputs are valid after the stream is synchronised."""
+    image and dL/dparams back, all enqueued by one C-ABI call (pdr_step_host):
+    the dL/dI upload and the image download overlap the render on a side
+    stream of the library that the current stream joins.  Returns (h_image,
+    h_grad_params, dev_bufs); the host outputs are valid after the current
+    stream is synchronised.  N = 0 (no Gaussians) gives a zero image."""
     if h_params.is_cuda or h_grad_image.is_cuda:
         raise ValueError("step_host takes host tensors")
     B, N, P = h_params.shape
