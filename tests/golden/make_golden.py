@@ -1,4 +1,5 @@
-"""Write tests/golden/tiny_oracle.txt from the fp64 oracle alone.
+"""Write tests/golden/tiny_oracle.txt and tests/golden/loss_oracle.txt from
+the fp64 oracle alone.
 
 The pages print no worked numeric example for the renderer, so this fixture is
 a regression lock on the oracle itself: the "tiny" workload (1 frame, C=1,
@@ -17,7 +18,31 @@ sys.path.insert(0, os.path.dirname(os.path.dirname(HERE)))
 import numpy as np  # noqa: E402
 
 import oracle  # noqa: E402
+from oracle import loss as oracle_loss  # noqa: E402
 from differentiable_gaussian_splatting_pdr_b200.inputs import WORKLOADS, make_inputs  # noqa: E402
+
+
+def loss_pair():
+    """The loss fixture's image / target pair: seeded draws, no arithmetic of
+    the method (image ~ U[0, 1), target = clip(image + N(0, 0.1)), fp32)."""
+    rng = np.random.default_rng(11)
+    x = rng.uniform(0, 1, (1, 2, 12, 17)).astype(np.float32)
+    y = np.clip(x + rng.normal(0, 0.1, x.shape), 0, 1).astype(np.float32)
+    return x, y
+
+
+def write_loss():
+    x, y = loss_pair()
+    loss, grad, (l1, ssim) = oracle_loss.l1_ssim_loss(x, y, 0.2)
+    path = os.path.join(HERE, "loss_oracle.txt")
+    with open(path, "w") as f:
+        f.write("# L1 + SSIM loss oracle (lam 0.2, range 1) on a seeded 1x2x12x17 pair\n")
+        f.write("# written by tests/golden/make_golden.py, which calls only oracle/\n")
+        f.write("loss %.17g\n" % loss)
+        f.write("l1 %.17g\n" % l1)
+        f.write("ssim %.17g\n" % ssim)
+        f.write("grad " + " ".join("%.17g" % v for v in grad.ravel()) + "\n")
+    print(path)
 
 
 def main():
@@ -39,3 +64,4 @@ def main():
 
 if __name__ == "__main__":
     main()
+    write_loss()

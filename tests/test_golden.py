@@ -31,3 +31,26 @@ def test_oracle_matches_golden_fixture():
     np.testing.assert_array_equal(ids, np.array(gold["tile_ids"], dtype=np.int32))
     np.testing.assert_array_equal(img.ravel(), np.array(gold["image"], dtype=np.float64))
     np.testing.assert_array_equal(grad.ravel(), np.array(gold["grad_params"], dtype=np.float64))
+
+
+LOSS_GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "loss_oracle.txt")
+
+
+def test_loss_oracle_matches_golden_fixture():
+    """The L1 + SSIM oracle on the fixture's seeded pair reproduces the stored
+    loss, its two terms and dL/dI (a regression lock on oracle/loss.py)."""
+    import sys
+    sys.path.insert(0, os.path.dirname(LOSS_GOLDEN))
+    from make_golden import loss_pair
+    from oracle import loss as oracle_loss
+    gold = {}
+    with open(LOSS_GOLDEN) as f:
+        for line in f:
+            if not line.startswith("#"):
+                key, *vals = line.split()
+                gold[key] = np.array(vals, dtype=np.float64)
+    x, y = loss_pair()
+    loss, grad, (l1, ssim) = oracle_loss.l1_ssim_loss(x, y, 0.2)
+    np.testing.assert_allclose([loss, l1, ssim], [gold["loss"][0], gold["l1"][0], gold["ssim"][0]],
+                               rtol=1e-14, atol=0)
+    np.testing.assert_allclose(grad.ravel(), gold["grad"], rtol=1e-12, atol=1e-18)
