@@ -142,6 +142,30 @@ def test_covariance_matrix_form(seed):
     assert np.abs(got - want).max() <= 1e-12 * scale
 
 
+def test_covariance_pin_catches_the_slips_it_targets():
+    """A rotation of the wrong sense, swapped scales, or a window one pixel too
+    small, planted in the independent reference, moves it far outside the
+    covariance pin's 1e-12 bar: the pin can tell the oracle from each slip."""
+    rng = np.random.default_rng(7)
+    B, N, C, H, W, k = 1, 9, 2, 21, 27, 9
+    p = np.empty((B, N, 5 + C), dtype=np.float32)
+    p[..., 0] = rng.uniform(4, W - 4, (B, N))
+    p[..., 1] = rng.uniform(4, H - 4, (B, N))
+    p[..., 2] = rng.normal(0.8, 0.3, (B, N))
+    p[..., 3] = p[..., 2] - 0.7                      # clearly anisotropic
+    p[..., 4] = rng.uniform(0.3, 1.2, (B, N))        # away from multiples of pi/2
+    p[..., 5:] = rng.normal(0, 1, (B, N, C))
+    got = oracle.render_fwd(p, H, W, k)
+    scale = np.abs(got).max()
+    flipped = p.copy()
+    flipped[..., 4] *= -1.0
+    swapped = p.copy()
+    swapped[..., [2, 3]] = p[..., [3, 2]]
+    for slip in (dense_reference(flipped, H, W, k), dense_reference(swapped, H, W, k),
+                 dense_reference(p, H, W, k - 2)):
+        assert np.abs(got - slip).max() > 1e-3 * scale
+
+
 def test_rotation_direction_on_diagonals():
     """theta = pi/4: the first axis (scale e^{s_1}) points along (1, 1) in (x, y)."""
     s1, s2 = 0.9, -0.2
