@@ -5,7 +5,10 @@ max|I_ref| per (frame, channel); gradients within 1e-4 of max|ref| per
 parameter field (mu_x, mu_y, s_1, s_2, theta, each a_c) per frame; tile
 binning bit-exact.  Inputs are the seeded workloads of inputs.py plus edge
 cases (ties at .5, off-grid and non-finite means, k = 1, windows spanning
-three tiles, ragged grids, odd widths, long lists, C up to 8).
+three tiles, ragged grids, odd widths, long lists, C up to 8, frames without
+Gaussians, the largest window with the largest C, a frame of the most tiles
+allowed), and the host-buffer step (back to back on one stream, and from two
+threads at once).
 """
 from __future__ import annotations
 
