@@ -183,3 +183,36 @@ def test_loss_workspace_sizes_and_validation_without_gpu():
         assert lib.pdr_loss_l1_ssim(*args) == _lib.STATUS_CODES["PDR_ERR_INVALID_ARG"], args
     assert lib.pdr_loss_l1_ssim(fake, fake, 1, 1, 8, 8, 0.2, 1.0, fake, fake, fake, 0, None) == \
         _lib.STATUS_CODES["PDR_ERR_WORKSPACE_TOO_SMALL"]
+
+
+def test_plain_c_caller(lib, tmp_path):
+    """include/pdr.h is plain C99 and libpdr.so is callable from C without
+    Python: a C program built against them runs the host-only entry points."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "caller.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include "pdr.h"
+int main(void) {
+    if (pdr_abi_version() != 1) return 1;
+    if (pdr_workspace_bytes(2, 64, 3, 40, 24, 9) == 0) return 2;
+    if (pdr_workspace_bytes(2, 64, 3, 40, 24, 8) != 0) return 3;      /* even k */
+    if (pdr_list_capacity_per_frame(100, 9) != 400) return 4;
+    if (pdr_render_fwd(NULL, 2, 64, 3, 40, 24, 9, NULL, NULL, 0, 0, NULL)
+        != PDR_ERR_INVALID_ARG) return 5;
+    printf("%s\n", pdr_status_string(PDR_ERR_TOO_LARGE));
+    return 0;
+}
+''')
+    exe = tmp_path / "caller"
+    libdir = os.path.dirname(_lib.LIB_PATH)
+    cc = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                         str(src), "-o", str(exe), "-L", libdir, "-lpdr", "-Wl,-rpath," + libdir],
+                        capture_output=True, text=True)
+    assert cc.returncode == 0, cc.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert run.returncode == 0, (run.returncode, run.stderr)
+    assert run.stdout.startswith("PDR_ERR_TOO_LARGE")
