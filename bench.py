@@ -40,7 +40,8 @@ from differentiable_gaussian_splatting_pdr_b200.inputs import (  # noqa: E402
 
 METRIC = "Gaussian-pixel evals/s and frames/s (fwd+bwd, 1 B200), % of roofline"
 UNIT = "evals/s"
-DEFAULT_WORKLOAD = "mono64"   # 16 frames, C=1, 64x64, N=1024/frame, k=9
+# The largest single-GPU workload: 8 frames, C=3, 512x512, N=65536/frame, k=15.
+DEFAULT_WORKLOAD = "stress512"
 SM_COUNT = 148
 FP32_LANES_PER_SM = 128
 L2_FLUSH_BYTES = 256 << 20
@@ -161,17 +162,26 @@ class ClockSampler:
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
+    def mark(self) -> int:
+        """Index of the next sample: summarise(a, b) covers samples between marks."""
+        return len(self.lines)
+
     def stop(self):
+        """Stop sampling; summary of every sample taken since start()."""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=5)
+        return self.summarise(0, None)
+
+    def summarise(self, a: int, b):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.thread.join(timeout=5)
         sm, mx, pw, reasons = [], [], [], set()
-        for line in self.lines:
+        for line in self.lines[a:b]:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
@@ -203,42 +213,59 @@ def oracle_sample(w, seconds: float, max_frames=None, threads=None):
     p, g = make_inputs(w)
     p, g = p[:B].copy(), g[:B].copy()
     ev = in_grid_evals(p, w.H, w.W, w.k)
-    cores = oracle.max_threads() if threads is None else max(1, int(threads))
+    threads = oracle.max_threads() if threads is None else max(1, int(threads))
+    cores = min(threads, B)  # OpenMP over frames: at most one thread per frame
     reps, t0 = 0, time.perf_counter()
     while True:
-        oracle.render_fwd(p, w.H, w.W, w.k, cores)
-        oracle.render_bwd(p, g, w.H, w.W, w.k, cores)
+        oracle.render_fwd(p, w.H, w.W, w.k, threads)
+        oracle.render_bwd(p, g, w.H, w.W, w.k, threads)
         reps += 1
         dt = time.perf_counter() - t0
         if dt >= seconds:
             break
-    sample = "%d x fwd+bwd of %d/%d frames of %s (%s)" % (reps, B, w.B, w.name, w.desc)
+    sample = ("%d x fwd+bwd of %d/%d frames of %s (%s), fp64 oracle, OpenMP over frames "
+              "on %d threads" % (reps, B, w.B, w.name, w.desc, cores))
     return ev * reps / dt, B * reps / dt, cores, sample, dt / reps
 
 
+REFERENCE_BUDGET_S = 150.0  # host-core seconds the whole reference arm may take
+
+
 def run_reference(args, w):
+    """The oracle as the reference arm: fp64 fwd + bwd on the host cores, on
+    whole batches of the workload (fewer frames per step only if K + W whole
+    batches would take longer than REFERENCE_BUDGET_S)."""
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return 0
-    import oracle
-    frames = w.B if w.name != "stress512" else 1
-    p, g = make_inputs(w)
-    p, g = p[:frames].copy(), g[:frames].copy()
+    import oracle  # test infrastructure: the reference arm is the oracle itself
+    threads = oracle.max_threads()
+    p_all, g_all = make_inputs(w)
+    t0 = time.perf_counter()
+    oracle.render_fwd(p_all, w.H, w.W, w.k, threads)
+    oracle.render_bwd(p_all, g_all, w.H, w.W, w.k, threads)
+    t_batch = time.perf_counter() - t0
+    frames = w.B
+    total = t_batch * (args.steps + args.warmup)
+    if total > REFERENCE_BUDGET_S:
+        frames = max(1, int(w.B * REFERENCE_BUDGET_S / total))
+    p, g = p_all[:frames].copy(), g_all[:frames].copy()
     ev = in_grid_evals(p, w.H, w.W, w.k)
-    cores = oracle.max_threads()
+    cores = min(threads, frames)
     for _ in range(args.warmup):
-        oracle.render_fwd(p, w.H, w.W, w.k, cores)
-        oracle.render_bwd(p, g, w.H, w.W, w.k, cores)
+        oracle.render_fwd(p, w.H, w.W, w.k, threads)
+        oracle.render_bwd(p, g, w.H, w.W, w.k, threads)
     times = []
     for _ in range(args.steps):
         t0 = time.perf_counter()
-        oracle.render_fwd(p, w.H, w.W, w.k, cores)
-        oracle.render_bwd(p, g, w.H, w.W, w.k, cores)
+        oracle.render_fwd(p, w.H, w.W, w.k, threads)
+        oracle.render_bwd(p, g, w.H, w.W, w.k, threads)
         times.append(time.perf_counter() - t0)
     tot = sum(times)
     value = ev * len(times) / tot
-    sample = "%d frames of %s per step (%s), fp64 oracle, OpenMP over frames" % (frames, w.name, w.desc)
+    sample = ("%d/%d frames of %s per step (%s), fp64 oracle, OpenMP over frames on %d threads"
+              % (frames, w.B, w.name, w.desc, cores))
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(times),
@@ -532,6 +559,7 @@ def run_gpu(args, w):
     gpu_id = "GPU-" + str(torch.cuda.get_device_properties(device).uuid).replace("GPU-", "")
     clocks = ClockSampler(gpu_id)
     clocks.start()
+    m0 = clocks.mark()  # the soak runs the timed step itself, so it counts as timed load
     t_soak = time.perf_counter()
     while time.perf_counter() - t_soak < args.soak:   # clocks settle under the same step
         flush.fill_(1)
@@ -547,7 +575,7 @@ def run_gpu(args, w):
     if world > 1:
         dist.barrier()
     # ----------------------------------------------
-    clk = clocks.stop()
+    m1 = clocks.mark()
     R.check_device_error(step.ws, device)
 
     eager = time_eager_steps(step, torch, flush, args.steps, stream)
@@ -605,6 +633,7 @@ def run_gpu(args, w):
             sp = time_graph(st, "split", flush, args.sweep_steps, stream)
             fs = time_graph(st, "fwd", flush, args.sweep_steps, stream)
             R.check_device_error(st.ws, device)
+            e2e_s, h2d_s, d2h_s = time_e2e_steps(st, torch, args.sweep_steps, stream)
             tot = float(pr[:, 0].mean())
             f_ms, b_ms = float(fs[:, 2].mean()), float(sp[:, 2].mean())
             of, ob = fp32_ops_per_eval(sw.C)
@@ -617,6 +646,9 @@ def run_gpu(args, w):
                 "fwd_frac": st.evals * of / (f_ms * 1e-3) / 1e12 / peak_tops,
                 "bwd_frac": st.evals * ob / (b_ms * 1e-3) / 1e12 / peak_tops,
                 "step_frac": st.evals * (of + ob) / (tot * 1e-3) / 1e12 / peak_tops,
+                "e2e": {"value": st.evals / (float(e2e_s.mean()) * 1e-3), "unit": UNIT,
+                        "h2d_bytes_per_step": h2d_s, "d2h_bytes_per_step": d2h_s,
+                        "api": "pdr_step_host"},
             }
             del st
             lbs = LossBench(R, torch, sw, sw.seed, device)
@@ -689,14 +721,25 @@ def run_gpu(args, w):
                            "step_frac": st.evals * (of + ob) / (tot * 1e-3) / 1e12 / peak_tops}
             del st
 
+    clk = clocks.stop()   # every GPU timed region of this run lies between start and here
+    clk_main = clocks.summarise(m0, m1)
+
     cpu = None
     if rank == 0 and world == 1 and args.cpu_seconds > 0:
         v, fps, cores, sample, _ = oracle_sample(w, args.cpu_seconds)
         cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
                "frames_per_s": fps}
-        v1, fps1, _, sample1, _ = oracle_sample(w, min(3.0, args.cpu_seconds), threads=1)
+        v1, fps1, _, sample1, _ = oracle_sample(w, min(3.0, args.cpu_seconds), max_frames=1,
+                                                threads=1)
         cpu["single_core"] = {"value": v1, "unit": UNIT, "cores": 1, "sample": sample1,
                               "frames_per_s": fps1}
+        # The oracle beside every other workload of the sweep (a bounded sample each).
+        for name in sweep:
+            sw = WORKLOADS[name]
+            ov, ofps, oc, osample, _ = oracle_sample(sw, min(2.0, args.cpu_seconds))
+            sweep[name]["cpu_baseline"] = {"value": ov, "unit": UNIT, "cores": oc,
+                                           "kind": "oracle", "sample": osample,
+                                           "frames_per_s": ofps}
 
     if rank == 0:
         launches_per_step = graph_kernel_nodes(step.graphs["main"])
@@ -724,6 +767,7 @@ def run_gpu(args, w):
                     "api": "pdr_step_host: pinned host -> device, fwd, bwd, device -> host"},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk,
+            "clocks_main_region": clk_main,
             "cpu_baseline": cpu,
             "loss_l1_ssim": loss_entry,
             "sweep": sweep,

@@ -39,6 +39,8 @@ SIGNATURES = {
     "pdr_step_host": (_i, [_vp, _vp, _vp, _vp] + [_i] * 6 + [_vp] * 5 + [_sz, _vp]),
     "pdr_check_device_error": (_i, [_vp, _vp]),
     "pdr_render_fwd_noalloc": (_i, [_vp] + [_i] * 6 + [_vp, _vp]),
+    "pdr_check_device_error_noalloc": (_i, [_vp]),
+    "pdr_workspace_part": (_i, [_i] * 7 + [ctypes.POINTER(_sz), ctypes.POINTER(_sz)]),
     "pdr_loss_workspace_bytes": (_sz, [_i] * 4),
     "pdr_render_fwd_ex": (_i, [_vp] + [_i] * 6 + [_vp, _i, _vp, _sz, _i, _vp]),
     "pdr_render_bwd_ex": (_i, [_vp, _vp, _i] + [_i] * 6 + [_vp, _vp, _sz, _i, _vp]),

@@ -149,6 +149,19 @@ def check_device_error(ws: Workspace, device=None) -> None:
                _lib.load().pdr_check_device_error(_ptr(ws.buf), _stream(device)))
 
 
+# Parts of the workspace (pdr_ws_part in include/pdr.h).
+WS_PARTS = {"error_word": 0, "records": 1, "tile_offsets": 2, "tile_ids": 3}
+
+
+def workspace_part(B: int, N: int, C: int, H: int, W: int, k: int, part: str):
+    """(byte offset, bytes) of a part of the workspace for these sizes."""
+    import ctypes
+    off, n = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    _lib.check("pdr_workspace_part", _lib.load().pdr_workspace_part(
+        B, N, C, H, W, k, WS_PARTS[part], ctypes.byref(off), ctypes.byref(n)))
+    return int(off.value), int(n.value)
+
+
 def bin_tiles(params: torch.Tensor, H: int, W: int, k: int):
     """Tile lists as the library builds them.
 
@@ -216,7 +229,11 @@ class _Render(torch.autograd.Function):
     def backward(ctx, grad_image):
         (params,) = ctx.saved_tensors
         H, W, k = ctx.hwk
-        grad = render_bwd(params, grad_image.float().contiguous(), H, W, k, ctx.ws, reuse_bins=True)
+        # fp16 / bf16 upstream gradients go to the library as they are (it
+        # widens each element to fp32 on load); other types become fp32.
+        if grad_image.dtype not in _DTYPES:
+            grad_image = grad_image.float()
+        grad = render_bwd(params, grad_image.contiguous(), H, W, k, ctx.ws, reuse_bins=True)
         ctx.ws = None
         return grad, None, None, None
 

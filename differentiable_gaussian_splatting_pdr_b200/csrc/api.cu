@@ -132,12 +132,18 @@ cudaError_t step_side(StepSide **out) {
     return cudaSuccess;
 }
 
+// Binning starts a new use of the workspace: the device error word is
+// cleared first, stream-ordered, so that no kernel of this call (or of a
+// render that reuses these bins) can have set a bit that the clear then wipes.
+cudaError_t clear_error_word(const Workspace &ws, cudaStream_t s) {
+    return cudaMemsetAsync(ws.err, 0, sizeof(int), s);
+}
+
 cudaError_t bin(const float *params, const Geom &g, const Workspace &ws, cudaStream_t s) {
-    if (g.N == 0) {  // no Gaussians: a clear error word and every tile list empty at 0
-        cudaError_t e = cudaMemsetAsync(ws.err, 0, sizeof(int), s);
-        if (e != cudaSuccess) return e;
+    cudaError_t e = clear_error_word(ws, s);
+    if (e != cudaSuccess) return e;
+    if (g.N == 0)  // no Gaussians: every tile list empty at 0
         return cudaMemsetAsync(ws.offs, 0, sizeof(int) * (size_t)g.B * (g.T + 1), s);
-    }
     return launch_bin(params, g, ws, s);
 }
 
@@ -221,8 +227,12 @@ pdr_status pdr_render_fwd_ex(const float *params, int B, int N, int C, int H, in
     g.img_dtype = image_dtype;
     g.out_vec2 = ((g.W & 1) == 0) && ((reinterpret_cast<uintptr_t>(image) & 7) == 0);
     g.out_vec4 = ((g.W & 3) == 0) && ((reinterpret_cast<uintptr_t>(image) & 15) == 0);
-    if (!workspace_holds_bins && g.cluster_fwd)  // small frames: bins + render, one launch
+    if (!workspace_holds_bins && g.cluster_fwd && fwd_cluster_schedulable(g)) {
+        // Small frames: bins + render in one clustered launch.
+        st = from_cuda(clear_error_word(ws, s));
+        if (st != PDR_OK) return st;
         return from_cuda(launch_fwd(params, g, ws, image, s, true));
+    }
     if (!workspace_holds_bins) {
         st = from_cuda(bin(params, g, ws, s));
         if (st != PDR_OK) return st;
@@ -287,8 +297,31 @@ pdr_status pdr_bin(const float *params, int B, int N, int C, int H, int W, int k
     st = from_cuda(cudaMemcpyAsync(tile_offsets, ws.offs, sizeof(int) * (size_t)g.B * (g.T + 1),
                                    cudaMemcpyDeviceToDevice, s));
     if (st != PDR_OK || g.cap == 0) return st;
-    return from_cuda(cudaMemcpyAsync(tile_ids, ws.ids, sizeof(int) * (size_t)g.B * g.cap,
-                                     cudaMemcpyDeviceToDevice, s));
+    // The lists as frame-local ids (the workspace copy also marks each
+    // Gaussian's home-tile entry for the backward pass).
+    return from_cuda(launch_copy_ids(tile_ids, ws.ids, (size_t)g.B * g.cap, s));
+}
+
+pdr_status pdr_workspace_part(int B, int N, int C, int H, int W, int k, int part,
+                              size_t *offset, size_t *bytes) {
+    Geom g;
+    pdr_status st = make_geom(B, N, C, H, W, k, &g);
+    if (st != PDR_OK) return st;
+    if (!offset || !bytes) return PDR_ERR_INVALID_ARG;
+    const Layout L = make_layout(g);
+    switch (part) {
+        case PDR_WS_ERROR_WORD: *offset = L.err; *bytes = sizeof(int); return PDR_OK;
+        case PDR_WS_RECORDS: *offset = L.gr; *bytes = L.hist - L.gr; return PDR_OK;
+        case PDR_WS_TILE_OFFSETS:
+            *offset = L.offs;
+            *bytes = sizeof(int) * (size_t)g.B * (g.T + 1);
+            return PDR_OK;
+        case PDR_WS_TILE_IDS:
+            *offset = L.ids;
+            *bytes = sizeof(int) * (size_t)g.B * g.cap;
+            return PDR_OK;
+        default: return PDR_ERR_INVALID_ARG;
+    }
 }
 
 pdr_status pdr_step_host(const float *h_params, const float *h_grad_image, float *h_image,

@@ -36,7 +36,6 @@ __global__ void __launch_bounds__(kCountThreads) k_count(const float *__restrict
                                                          int *__restrict__ err) {
     extern __shared__ int hs[];  // [T]
     const int b = blockIdx.y, c = blockIdx.x;
-    if (b == 0 && c == 0 && threadIdx.x == 0) *err = 0;
     for (int t = threadIdx.x; t < g.T; t += blockDim.x) hs[t] = 0;
     __syncthreads();
     const int i0 = c * kBinChunk, i1 = min(i0 + kBinChunk, g.N);
@@ -174,11 +173,13 @@ __global__ void k_scatter(Geom g, const float4 *__restrict__ gr, const int *__re
     for (int s = i0; s < i1; s += blockDim.x) {
         const int i = s + threadIdx.x;
         int tx0 = 1, tx1 = 0, ty0 = 1, ty1 = 0;  // empty unless the window hits the grid
+        int ht = -1;                              // home tile
         if (i < i1) {
             const float4 Q = gr[2 * ((size_t)b * g.N + i) + 1];
             int x0, x1, y0, y1;
             if (window_rect(__float_as_int(Q.z), __float_as_int(Q.w), g, x0, x1, y0, y1)) {
                 tx0 = x0 >> 4; tx1 = x1 >> 4; ty0 = y0 >> 4; ty1 = y1 >> 4;
+                ht = home_tile(__float_as_int(Q.z), __float_as_int(Q.w), g);
             }
         }
         for (int ty = ty0; ty <= ty1; ++ty)
@@ -191,7 +192,7 @@ __global__ void k_scatter(Geom g, const float4 *__restrict__ gr, const int *__re
                 for (int w = 0; w < warp; ++w) pre += __popc(masks[w * g.T + t]);
                 const long long slot = (long long)base_s[t] + pre;
                 if (slot >= lo && slot < hi)
-                    ids[slot] = i;
+                    ids[slot] = (int)((unsigned)i | (t == ht ? kHomeFlag : 0u));
                 else
                     atomicOr(err, kErrListBounds);
             }
@@ -224,7 +225,6 @@ __global__ void __launch_bounds__(1024) k_bin_frame(const float *__restrict__ pa
     __shared__ int warp_tot[32];
     const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const unsigned lt = lanemask_lt();
-    if (b == 0 && tid == 0) *err = 0;
     for (int t = tid; t < T; t += blockDim.x) run[t] = 0;
     for (int t = tid; t < nw * T; t += blockDim.x) masks[t] = 0u;
     __syncthreads();
@@ -278,11 +278,13 @@ __global__ void __launch_bounds__(1024) k_bin_frame(const float *__restrict__ pa
     for (int s = 0; s < g.N; s += blockDim.x) {
         const int i = s + tid;
         int tx0 = 1, tx1 = 0, ty0 = 1, ty1 = 0;  // empty unless the window hits the grid
+        int ht = -1;                              // home tile
         if (i < g.N) {
             const float4 Q = gr[2 * ((size_t)b * g.N + i) + 1];
             int x0, x1, y0, y1;
             if (window_rect(__float_as_int(Q.z), __float_as_int(Q.w), g, x0, x1, y0, y1)) {
                 tx0 = x0 >> 4; tx1 = x1 >> 4; ty0 = y0 >> 4; ty1 = y1 >> 4;
+                ht = home_tile(__float_as_int(Q.z), __float_as_int(Q.w), g);
             }
         }
         for (int ty = ty0; ty <= ty1; ++ty)
@@ -303,7 +305,7 @@ __global__ void __launch_bounds__(1024) k_bin_frame(const float *__restrict__ pa
                 const long long slot =
                     (long long)run[t] + pre[warp * T + t] + __popc(my[t] & lt);
                 if (slot >= lo && slot < hi)
-                    ids[slot] = i;
+                    ids[slot] = (int)((unsigned)i | (t == ht ? kHomeFlag : 0u));
                 else
                     atomicOr(err, kErrListBounds);
             }
@@ -316,7 +318,20 @@ __global__ void __launch_bounds__(1024) k_bin_frame(const float *__restrict__ pa
     }
 }
 
+__global__ void k_copy_ids(int *__restrict__ dst, const int *__restrict__ src, size_t n) {
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (size_t)gridDim.x * blockDim.x)
+        dst[i] = entry_id(src[i]);
+}
+
 }  // namespace
+
+cudaError_t launch_copy_ids(int *dst, const int *src, size_t n, cudaStream_t s) {
+    if (n == 0) return cudaSuccess;
+    const size_t blocks = (n + 255) / 256;
+    k_copy_ids<<<(unsigned)(blocks < 4 * 148 ? blocks : 4 * 148), 256, 0, s>>>(dst, src, n);
+    return cudaGetLastError();
+}
 
 size_t bin_frame_smem(const Geom &g) {
     return sizeof(int) * (size_t)g.T * (2 + 2 * (g.frame_threads / 32));

@@ -18,6 +18,14 @@ constexpr int kErrListBounds = 1;  // a tile list or list slot outside its frame
 constexpr int kErrBadId = 2;       // a list entry that is not a Gaussian of the frame
 constexpr int kErrSmemLayout = 4;  // a kernel got less dynamic shared memory than it lays out
 
+// A tile-list entry is a frame-local Gaussian id; the binner sets kHomeFlag on
+// the one entry of each Gaussian that sits in the list of its home tile (the
+// tile of its clamped window centre), so that the backward pass finds its
+// Gaussians from the ids alone.
+constexpr unsigned kHomeFlag = 0x80000000u;
+__device__ __forceinline__ int entry_id(int raw) { return raw & 0x7fffffff; }
+__device__ __forceinline__ bool entry_home(int raw) { return raw < 0; }
+
 // sqrt(kappa) with kappa = log2(e) / 2: scaling u by sqrt(kappa e^{-2 s})
 // turns exp(-q / 2) into 2^{-(u1^2 + u2^2)}.
 constexpr float kSqrtKappa = 0.849321800288019f;
@@ -199,10 +207,18 @@ cudaError_t launch_fwd(const float *params, const Geom &g, const Workspace &ws,
 cudaError_t launch_bwd(const float *params, const void *grad_image, const Geom &g,
                        const Workspace &ws, float *grad_params, cudaStream_t s);
 
+// The fused bins + render launch (k_fwd_cluster) for these sizes can be
+// scheduled on the current device (at least one cluster fits); cached.
+bool fwd_cluster_schedulable(const Geom &g);
+// dst[i] = frame-local id of tile-list entry src[i] (home flag cleared).
+cudaError_t launch_copy_ids(int *dst, const int *src, size_t n, cudaStream_t s);
+
 // Dynamic shared memory needed by the kernels for these sizes.
 size_t bin_frame_smem(const Geom &g);
 size_t bin_count_smem(const Geom &g);
 size_t bin_scatter_smem(const Geom &g);
 size_t bwd_smem(const Geom &g);
+size_t bwd_smem_nt(const Geom &g, int nt);
+int bwd_threads(const Geom &g);  // threads per block of the scalar backward
 
 }  // namespace pdr

@@ -56,7 +56,15 @@ extern "C" pdr_status pdr_render_fwd_noalloc(const float *params, int B, int N, 
     if (scratch_address(&scratch) != cudaSuccess) return PDR_ERR_CUDA;
     // The bins are rebuilt on every call, and every word of the scratch that
     // the kernels read is written earlier in the same call (the error word is
-    // reset by the first kernel), so the previous call's leftovers never leak.
+    // cleared before the first kernel), so the previous call's leftovers never
+    // leak.
     return pdr_render_fwd(params, B, N, C, H, W, k, image, scratch, PDR_STATIC_SCRATCH_BYTES,
                           /*workspace_holds_bins=*/0, stream);
+}
+
+extern "C" pdr_status pdr_check_device_error_noalloc(void *stream) {
+    void *scratch = nullptr;
+    if (scratch_address(&scratch) != cudaSuccess) return PDR_ERR_CUDA;
+    // The error word is the first word of any workspace layout.
+    return pdr_check_device_error(scratch, stream);
 }

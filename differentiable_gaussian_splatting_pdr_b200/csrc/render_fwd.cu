@@ -28,6 +28,10 @@
 // shared memory; then every block renders its tile from its own list.
 #include <cooperative_groups.h>
 
+#include <map>
+#include <mutex>
+#include <tuple>
+
 #include "common.cuh"
 
 namespace cg = cooperative_groups;
@@ -60,7 +64,23 @@ struct FwdSmem {
     unsigned win[NB];  // window as column bits | row bits << 16 (tile pixels)
     unsigned sub[16][NB];
     int subn[16];
+    // pen[m].j = 0 if bit j of m is set, else +inf: added to the quadratic
+    // form of a lane's pixel j, it turns the weight of a pixel outside the
+    // window into 2^-inf = 0 without a branch or a predicate per pixel.
+    float4 pen[16];
 };
+
+__device__ __forceinline__ float2 f2fma(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+
+template <int C, int NB>
+__device__ __forceinline__ void init_pen(FwdSmem<C, NB> &S) {
+    if (threadIdx.x < 16) {
+        const float inf = __int_as_float(0x7f800000);
+        const unsigned m = threadIdx.x;
+        S.pen[m] = make_float4(m & 1u ? 0.0f : inf, m & 2u ? 0.0f : inf, m & 4u ? 0.0f : inf,
+                               m & 8u ? 0.0f : inf);
+    }
+}
 
 // Render the entries list[0 .. L) (frame-local ids, ascending) of the tile at
 // (X0, Y0) of frame b into acc.  Called by the whole block.
@@ -69,7 +89,7 @@ struct FwdSmem {
 template <int C, int PL, int NB, typename Fetch>
 __device__ __forceinline__ void render_list(const Geom &g, Fetch fetch, const int *list,
                                             int L, int X0, int Y0, int *err,
-                                            FwdSmem<C, NB> &S, float (&acc)[PL][C]) {
+                                            FwdSmem<C, NB> &S, float2 (&acc)[PL / 2][C]) {
     using LY = FwdLayout<PL>;
     constexpr int RV = FwdRec<C>::kVec;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -85,8 +105,8 @@ __device__ __forceinline__ void render_list(const Geom &g, Fetch fetch, const in
         const int n = min(NB, L - e0);
         __syncthreads();  // the previous batch is fully consumed
         for (int e = tid; e < n; e += LY::kThreads) {
-            const int i = list[e0 + e];
-            if ((unsigned)i >= (unsigned)g.N) {  // never for consistent bins
+            const int i = entry_id(list[e0 + e]);
+            if (i >= g.N) {  // never for consistent bins
                 atomicOr(err, kErrBadId);
                 S.win[e] = 0u;
                 continue;
@@ -152,6 +172,10 @@ __device__ __forceinline__ void render_list(const Geom &g, Fetch fetch, const in
         __syncthreads();
         const int ns = S.subn[grp];
         const unsigned *sl = S.sub[grp];
+        // Pixel pairs (x, x + 1) of the lane's run with the packed f32x2
+        // arithmetic of sm_100: one instruction per pair for each step of the
+        // quadratic form and each channel's accumulation.  A pixel outside the
+        // window gets +inf added to its quadratic form (weight exactly 0).
         for (int s = 0; s < ns; ++s) {
             const unsigned pk = sl[s];
             const float4 *r4 = reinterpret_cast<const float4 *>(
@@ -162,20 +186,23 @@ __device__ __forceinline__ void render_list(const Geom &g, Fetch fetch, const in
                 const float4 q = r4[v];
                 rr[4 * v] = q.x; rr[4 * v + 1] = q.y; rr[4 * v + 2] = q.z; rr[4 * v + 3] = q.w;
             }
-            const unsigned bits = pk >> bitshift;
-            float u1 = fmaf(rr[0], fx, fmaf(rr[1], fy, rr[2]));
-            float u2 = fmaf(rr[3], fx, fmaf(rr[4], fy, rr[5]));
+            const float4 P = S.pen[(pk >> bitshift) & 0xfu];
+            const float a1 = rr[0], a2 = rr[3];
+            const float u1 = fmaf(a1, fx, fmaf(rr[1], fy, rr[2]));
+            const float u2 = fmaf(a2, fx, fmaf(rr[4], fy, rr[5]));
+            float2 U1 = make_float2(u1, u1 + a1), U2 = make_float2(u2, u2 + a2);
 #pragma unroll
-            for (int j = 0; j < PL; ++j) {
-                if (j) {
-                    u1 += rr[0];
-                    u2 += rr[3];
+            for (int h = 0; h < PL / 2; ++h) {
+                if (h) {
+                    const float d1 = a1 + a1, d2 = a2 + a2;
+                    U1 = make_float2(U1.x + d1, U1.y + d1);
+                    U2 = make_float2(U2.x + d2, U2.y + d2);
                 }
-                const float w = ex2(fmaf(-u1, u1, -u2 * u2));
-                if (bits & (1u << j)) {
+                const float2 pen = h ? make_float2(P.z, P.w) : make_float2(P.x, P.y);
+                const float2 q = f2fma(U1, U1, f2fma(U2, U2, pen));
+                const float2 w = make_float2(ex2(-q.x), ex2(-q.y));
 #pragma unroll
-                    for (int c = 0; c < C; ++c) acc[j][c] = fmaf(rr[6 + c], w, acc[j][c]);
-                }
+                for (int c = 0; c < C; ++c) acc[h][c] = f2fma(make_float2(rr[6 + c], rr[6 + c]), w, acc[h][c]);
             }
         }
     }
@@ -183,7 +210,15 @@ __device__ __forceinline__ void render_list(const Geom &g, Fetch fetch, const in
 
 template <int C, int PL>
 __device__ __forceinline__ void store_tile(const Geom &g, int b, int X0, int Y0,
-                                           void *__restrict__ image_, const float (&acc)[PL][C]) {
+                                           void *__restrict__ image_, const float2 (&acc2)[PL / 2][C]) {
+    float acc[PL][C];
+#pragma unroll
+    for (int h = 0; h < PL / 2; ++h)
+#pragma unroll
+        for (int c = 0; c < C; ++c) {
+            acc[2 * h][c] = acc2[h][c].x;
+            acc[2 * h + 1][c] = acc2[h][c].y;
+        }
     using LY = FwdLayout<PL>;
     const int tid = threadIdx.x;
     const int grp = tid / LY::kLanes, lig = tid % LY::kLanes;
@@ -230,11 +265,12 @@ __global__ void __launch_bounds__(FwdLayout<PL>::kThreads) k_fwd(const float *__
     const int b = blockIdx.x / g.T, t = blockIdx.x - b * g.T;
     const int ty = t / g.TX, tx = t - ty * g.TX;
     const int X0 = tx * kTile, Y0 = ty * kTile;
-    float acc[PL][C];
+    float2 acc[PL / 2][C];
 #pragma unroll
-    for (int j = 0; j < PL; ++j)
+    for (int j = 0; j < PL / 2; ++j)
 #pragma unroll
-        for (int c = 0; c < C; ++c) acc[j][c] = 0.0f;
+        for (int c = 0; c < C; ++c) acc[j][c] = make_float2(0.0f, 0.0f);
+    init_pen(S);
     int L0, L1;
     list_range(offs, g, b, t, err, L0, L1);
     auto fetch = [&](int i, float4 &A, float4 &Q, float (&amp)[C]) {
@@ -273,9 +309,9 @@ __global__ void __launch_bounds__(FwdLayout<PL>::kThreads) k_fwd_cluster(
     const int b = blockIdx.y;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const unsigned lt = lanemask_lt();
-    if (b == 0 && q == 0 && tid == 0) *err = 0;
     if (tid < kClusterTiles) cnt[tid] = 0;
     if (tid < NW * kClusterTiles) masks[tid / kClusterTiles][tid % kClusterTiles] = 0u;
+    init_pen(S);
     __syncthreads();
 
     // 1. records and per-tile counts of this block's chunk
@@ -340,11 +376,13 @@ __global__ void __launch_bounds__(FwdLayout<PL>::kThreads) k_fwd_cluster(
     for (int s = i0; s < i1; s += NT) {
         const int i = s + tid;
         int tx0 = 1, tx1 = 0, ty0 = 1, ty1 = 0;
+        int ht = -1;  // home tile
         if (i < i1) {
             const float4 Q = gr[2 * ((size_t)b * g.N + i) + 1];
             int x0, x1, y0, y1;
             if (window_rect(__float_as_int(Q.z), __float_as_int(Q.w), g, x0, x1, y0, y1)) {
                 tx0 = x0 >> 4; tx1 = x1 >> 4; ty0 = y0 >> 4; ty1 = y1 >> 4;
+                ht = home_tile(__float_as_int(Q.z), __float_as_int(Q.w), g);
             }
         }
         for (int yy = ty0; yy <= ty1; ++yy)
@@ -357,7 +395,7 @@ __global__ void __launch_bounds__(FwdLayout<PL>::kThreads) k_fwd_cluster(
                 for (int w = 0; w < warp; ++w) pre += __popc(masks[w][tt]);
                 const long long slot = (long long)frame0 + pre;
                 if (slot >= lo && slot < hi) {
-                    ids[slot] = i;
+                    ids[slot] = (int)((unsigned)i | (tt == ht ? kHomeFlag : 0u));
                     const int local = pre - tstart[tt];
                     if (local < kClusterListCap) *cluster.map_shared_rank(list + local, tt) = i;
                 } else {
@@ -379,11 +417,11 @@ __global__ void __launch_bounds__(FwdLayout<PL>::kThreads) k_fwd_cluster(
     // 4. render this tile from its own list
     const int ty = q / g.TX, tx = q - ty * g.TX;
     const int X0 = tx * kTile, Y0 = ty * kTile;
-    float acc[PL][C];
+    float2 acc[PL / 2][C];
 #pragma unroll
-    for (int j = 0; j < PL; ++j)
+    for (int j = 0; j < PL / 2; ++j)
 #pragma unroll
-        for (int c = 0; c < C; ++c) acc[j][c] = 0.0f;
+        for (int c = 0; c < C; ++c) acc[j][c] = make_float2(0.0f, 0.0f);
     const int L = tstart[q + 1] - tstart[q];
     const int *src = L <= kClusterListCap ? list : ids + frame0 + tstart[q];
     if (onchip) {
@@ -440,6 +478,39 @@ cudaError_t launch_fwd_cluster(const float *params, const Geom &g, const Workspa
         return cudaGetLastError();
 }
 
+// At least one cluster of g.T blocks of k_fwd_cluster<C, PL> fits on the
+// current device (a cluster of more than 8 blocks needs the non-portable size).
+template <int C, int PL>
+bool cluster_fits(const Geom &g) {
+    if (g.T > 8 && cudaFuncSetAttribute(k_fwd_cluster<C, PL>,
+                                        cudaFuncAttributeNonPortableClusterSizeAllowed,
+                                        1) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    cfg.gridDim = dim3(g.T, 1, 1);
+    cfg.blockDim = dim3(FwdLayout<PL>::kThreads, 1, 1);
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = g.T;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, k_fwd_cluster<C, PL>, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return n > 0;
+}
+
+template <int C>
+bool cluster_fits_c(const Geom &g) {
+    return g.fwd_pl == 2 ? cluster_fits<C, 2>(g) : cluster_fits<C, 4>(g);
+}
+
 template <int C>
 cudaError_t launch_fwd_c(const float *params, const Geom &g, const Workspace &ws, void *image,
                          cudaStream_t s, bool bin_inside) {
@@ -456,6 +527,31 @@ cudaError_t launch_fwd_c(const float *params, const Geom &g, const Workspace &ws
 }
 
 }  // namespace
+
+bool fwd_cluster_schedulable(const Geom &g) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    static std::mutex mu;
+    static std::map<std::tuple<int, int, int, int>, bool> known;  // (device, C, PL, T)
+    const auto key = std::make_tuple(dev, g.C, g.fwd_pl, g.T);
+    std::lock_guard<std::mutex> lock(mu);
+    const auto it = known.find(key);
+    if (it != known.end()) return it->second;
+    bool ok = false;
+    switch (g.C) {
+        case 1: ok = cluster_fits_c<1>(g); break;
+        case 2: ok = cluster_fits_c<2>(g); break;
+        case 3: ok = cluster_fits_c<3>(g); break;
+        case 4: ok = cluster_fits_c<4>(g); break;
+        case 5: ok = cluster_fits_c<5>(g); break;
+        case 6: ok = cluster_fits_c<6>(g); break;
+        case 7: ok = cluster_fits_c<7>(g); break;
+        case 8: ok = cluster_fits_c<8>(g); break;
+        default: ok = false;
+    }
+    known[key] = ok;
+    return ok;
+}
 
 cudaError_t launch_fwd(const float *params, const Geom &g, const Workspace &ws, void *image,
                        cudaStream_t s, bool bin_inside) {

@@ -155,11 +155,19 @@ def knob_workloads(base: str = "mono64"):
                                       desc=w.desc + ", grid-initialised means")}
     for n in (w.N // 4, w.N * 4):
         out["%s-N%d" % (base, n)] = replace(w, N=n, name="%s-N%d" % (base, n),
-                                              desc="%s with N=%d" % (w.desc, n))
+                                              desc=_desc(w, N=n))
     for k in (5, 13, 17):
         out["%s-k%d" % (base, k)] = replace(w, k=k, name="%s-k%d" % (base, k),
-                                              desc="%s with k=%d" % (w.desc, k))
+                                              desc=_desc(w, k=k))
     return out
+
+
+def _desc(w: Workload, **kw) -> str:
+    """Description of workload w with some of its sizes replaced."""
+    v = replace(w, **kw)
+    amp = {"normal": "a~N(%g,%g)", "exponential": "a~Exp(%g)"}[v.amp[0]]
+    amp = amp % ((v.amp[1],) if v.amp[0] == "exponential" else (v.amp[1], v.amp[2]))
+    return "%d frames, C=%d, %dx%d, N=%d/frame, k=%d, %s" % (v.B, v.C, v.H, v.W, v.N, v.k, amp)
 
 
 def rank_seed(w: Workload, rank: int) -> int:

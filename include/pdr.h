@@ -179,11 +179,20 @@ pdr_status pdr_step_host(const float *h_params, const float *h_grad_image,
  *     device address (cudaGetSymbolAddress) and caches it; make that first
  *     call before any stream capture.
  *   - All calls on a device share the one scratch, which keeps the last
- *     call's contents.  Each call rebuilds everything it reads, so nothing
+ *     call's contents.  Each call rebuilds everything it reads (its device
+ *     error word included, cleared before its first kernel), so nothing
  *     needs clearing, but calls that overlap on the GPU (other streams, other
- *     host threads) race on it: serialise them. */
+ *     host threads) race on it: serialise them.
+ *   - The kernels' own bounds checks report into that scratch's error word;
+ *     pdr_check_device_error_noalloc reads it. */
 pdr_status pdr_render_fwd_noalloc(const float *params, int B, int N, int C, int H,
                                   int W, int k, float *image, void *stream);
+
+/* pdr_check_device_error for the built-in scratch of pdr_render_fwd_noalloc
+ * on the current device: synchronises `stream`, returns PDR_ERR_INTERNAL if a
+ * kernel's bounds check fired since the last call of pdr_render_fwd_noalloc
+ * began, and clears the word.  Allocates nothing. */
+pdr_status pdr_check_device_error_noalloc(void *stream);
 
 /* ---- Reduced-precision image storage ------------------------------------------
  * Image and dL/dI stored as fp16 or bf16 (half the bytes of the two largest
@@ -212,8 +221,30 @@ pdr_status pdr_render_bwd_ex(const float *params, const void *grad_image, int gr
 
 /* Synchronises `stream` and reports the device-side error word in the
  * workspace (PDR_ERR_INTERNAL if a kernel's own bounds check fired), then
- * clears it. */
+ * clears it.  The word is also cleared, stream-ordered, by every call that
+ * bins (pdr_build_bins, pdr_bin, and the render calls with their
+ * workspace_holds_*bins flag at 0) before its first kernel; kernels only ever
+ * set bits in it, so a bit set by any kernel since the last binning stays set
+ * until it is read here. */
 pdr_status pdr_check_device_error(void *workspace, void *stream);
+
+/* Where a part of the workspace lies, for tools and tests that inspect or
+ * plant values in it: byte offset from the workspace start and size in bytes
+ * of part `part` (a pdr_ws_part) for these sizes.  The tile offsets are
+ * int32 [B][T + 1] absolute list positions (as pdr_bin returns them); the
+ * tile ids are int32 [B * cap] entries whose bit 31 marks the one entry of
+ * each Gaussian in the list of its home tile (the tile of its window centre
+ * clamped to the grid), bits 0..30 the frame-local id.  Returns
+ * PDR_ERR_INVALID_ARG for an unknown part or null outputs, and the sizes'
+ * own validation errors. */
+typedef enum {
+    PDR_WS_ERROR_WORD = 0,
+    PDR_WS_RECORDS = 1,
+    PDR_WS_TILE_OFFSETS = 2,
+    PDR_WS_TILE_IDS = 3
+} pdr_ws_part;
+pdr_status pdr_workspace_part(int B, int N, int C, int H, int W, int k, int part,
+                              size_t *offset, size_t *bytes);
 
 /* ---- Training loss: L1 + SSIM, producing dL/dI ------------------------------
  * The objective the reading notes (section "Method", third point; "Key

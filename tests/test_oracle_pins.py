@@ -426,3 +426,38 @@ def test_grid_layout_puts_one_gaussian_per_cell():
     cell = np.floor(my / (w.H / gy)) * gx + np.floor(mx / (w.W / gx))
     for b in range(w.B):
         assert np.array_equal(np.sort(cell[b]), np.arange(w.N))
+
+
+@pytest.mark.parametrize("H,W,k,seed", [(40, 56, 17, 1), (23, 37, 21, 2), (64, 64, 9, 3), (7, 9, 3, 4)])
+def test_binning_matches_a_python_rect_test(H, W, k, seed):
+    """The oracle's tile lists against a rect test written here from the
+    definition alone (window = k x k pixels centred on round(mu) with ties up,
+    clipped to the grid; a Gaussian enters every 16 x 16 tile the clipped
+    window touches, ids ascending), sharing no code with the oracle."""
+    import math
+    rng = np.random.default_rng(seed)
+    N = 60
+    p = np.zeros((1, N, 6), dtype=np.float32)
+    p[0, :, 0] = rng.uniform(-k, W + k, N)
+    p[0, :, 1] = rng.uniform(-k, H + k, N)
+    p[0, :6, 0] = [0.5, 15.5, np.nextafter(np.float32(16.5), np.float32(0)), -0.5, W - 0.5, np.nan]
+    p[0, :, 2:4] = 0.5
+    p[0, :, 5] = 1.0
+    offs, ids = oracle.bin_tiles(p, H, W, k)
+    r = (k - 1) // 2
+    TX, TY = (W + 15) // 16, (H + 15) // 16
+    want = [[] for _ in range(TX * TY)]
+    for i in range(N):
+        mx, my = float(p[0, i, 0]), float(p[0, i, 1])
+        if not (math.isfinite(mx) and math.isfinite(my)):
+            continue
+        cx, cy = math.floor(mx + 0.5), math.floor(my + 0.5)  # exact: fp32 + 0.5 in fp64
+        x0, x1 = max(cx - r, 0), min(cx + r, W - 1)
+        y0, y1 = max(cy - r, 0), min(cy + r, H - 1)
+        if x0 > x1 or y0 > y1:
+            continue
+        for ty in range(y0 // 16, y1 // 16 + 1):
+            for tx in range(x0 // 16, x1 // 16 + 1):
+                want[ty * TX + tx].append(i)
+    got = [ids[offs[t]:offs[t + 1]].tolist() for t in range(TX * TY)]
+    assert got == want

@@ -2,7 +2,8 @@
 device memory (for example a plugin whose host application owns all device
 memory, or a loop that must not allocate after start-up).  It uses a scratch
 array built into the library instead of a caller workspace; its output must
-match the workspace entry point pdr_render_fwd, call after call.
+match the workspace entry point pdr_render_fwd, call after call, and the
+fp64 oracle; repeated calls must leave the device's free memory unchanged.
 
 This file is collected last on purpose, so that a failure here comes after
 every other test has run.
@@ -11,6 +12,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from differentiable_gaussian_splatting_pdr_b200 import _lib
 from differentiable_gaussian_splatting_pdr_b200 import api as R
 from differentiable_gaussian_splatting_pdr_b200 import build as pdr_build
@@ -86,3 +88,27 @@ def test_noalloc_frame_without_gaussians(lib):
     p = torch.zeros((2, 0, 7), device="cuda")
     got = _noalloc(lib, p, 40, 24, 9)
     assert got.shape == (2, 2, 40, 24) and not got.any()
+
+
+def test_noalloc_matches_the_oracle(lib):
+    w = WORKLOADS["rgb128"].scaled(B=3)
+    p_np = make_params(w, 11)
+    got = _noalloc(lib, torch.from_numpy(p_np).cuda(), w.H, w.W, w.k)
+    ref = oracle.render_fwd(p_np, w.H, w.W, w.k, max(1, oracle.max_threads()))
+    assert _normwise(got, ref) <= FWD_TOL
+
+
+def test_noalloc_allocates_nothing_and_reports_device_errors(lib):
+    """After the first call, further calls leave the device's free memory as it
+    was; the scratch's device error word reads back clear."""
+    w = WORKLOADS["mono64"]
+    p = torch.from_numpy(make_params(w, 3)).cuda()
+    out = torch.empty((w.B, w.C, w.H, w.W), device="cuda")
+    args = (p.data_ptr(), w.B, w.N, w.C, w.H, w.W, w.k, out.data_ptr(), _stream())
+    _lib.check("pdr_render_fwd_noalloc", lib.pdr_render_fwd_noalloc(*args))
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    for _ in range(3):
+        _lib.check("pdr_render_fwd_noalloc", lib.pdr_render_fwd_noalloc(*args))
+    _lib.check("pdr_check_device_error_noalloc", lib.pdr_check_device_error_noalloc(_stream()))
+    assert torch.cuda.mem_get_info()[0] == free0
