@@ -42,9 +42,9 @@ pdr_status make_geom(int B, int N, int C, int H, int W, int k, Geom *g) {
     g->m = (int)m;
     g->cap = (int)cap;
     g->nchunks = (N + kBinChunk - 1) / kBinChunk;
-    int nw = kScatterWarps;  // scatter block: as many warps as the per-warp tile masks allow
-    while (nw > 1 && sizeof(int) * (size_t)T * (nw + 2) > kScatterSmemLimit) nw >>= 1;
-    if (sizeof(int) * (size_t)T * (nw + 2) > kScatterSmemLimit) return PDR_ERR_TOO_LARGE;
+    int nw = kScatterWarps;  // scatter block: as many warps as the per-warp tile tables allow
+    while (nw > 1 && (size_t)T * (6 * nw + 4) + 16 > kScatterSmemLimit) nw >>= 1;
+    if ((size_t)T * (6 * nw + 4) + 16 > kScatterSmemLimit) return PDR_ERR_TOO_LARGE;
     g->scatter_warps = nw;
     // Small frames: one binning block per frame (its shared-memory tables
     // hold [2 + 2 * warps] x T ints).
@@ -65,13 +65,27 @@ pdr_status make_geom(int B, int N, int C, int H, int W, int k, Geom *g) {
     g->out_vec2 = 0;
     g->out_vec4 = 0;
     g->img_dtype = PDR_F32;
+    // Backward record capacity: room for the home Gaussians of a tile at 1.5x
+    // the mean count (a tile with more is processed in several rounds), at
+    // least one block's worth of list entries, at most 512.
+    // The pixel-pair kernel runs 128-thread blocks (short last rounds of its
+    // 16 groups per tile); the scalar kernel 256-thread blocks (measured on B200).
+    {
+        const long long mean = ((long long)N + T - 1) / T;
+        long long cap = ((mean * 3 / 2 + 32 + 31) / 32) * 32;
+        const int nt = bwd_uses_pairs(C, k) ? 128 : 256;
+        if (cap < nt) cap = nt;
+        if (cap > 512) cap = 512;
+        g->bwd_threads = nt;
+        g->bwd_rcap = (int)cap;
+    }
     return PDR_OK;
 }
 
 Layout make_layout(const Geom &g) {
     Layout L;
     size_t o = 0;
-    L.err = o; o += align_up(sizeof(int));
+    L.err = o; o += align_up(sizeof(int) * (1 + (size_t)g.B));  // error word, then the scan counters
     L.gr = o; o += align_up(sizeof(float4) * 2 * (size_t)g.B * g.N);
     L.hist = o; o += align_up(sizeof(int) * (size_t)g.B * g.nchunks * g.T);
     L.offs = o; o += align_up(sizeof(int) * (size_t)g.B * (g.T + 1));
@@ -84,6 +98,7 @@ Workspace carve(void *base, const Layout &L) {
     char *p = static_cast<char *>(base);
     Workspace w;
     w.err = reinterpret_cast<int *>(p + L.err);
+    w.done = w.err + 1;
     w.gr = reinterpret_cast<float4 *>(p + L.gr);
     w.hist = reinterpret_cast<int *>(p + L.hist);
     w.offs = reinterpret_cast<int *>(p + L.offs);
@@ -139,8 +154,13 @@ cudaError_t clear_error_word(const Workspace &ws, cudaStream_t s) {
     return cudaMemsetAsync(ws.err, 0, sizeof(int), s);
 }
 
+// The error word and the tile scan's per-frame counters, cleared together.
+cudaError_t clear_error_and_counters(const Geom &g, const Workspace &ws, cudaStream_t s) {
+    return cudaMemsetAsync(ws.err, 0, sizeof(int) * (1 + (size_t)g.B), s);
+}
+
 cudaError_t bin(const float *params, const Geom &g, const Workspace &ws, cudaStream_t s) {
-    cudaError_t e = clear_error_word(ws, s);
+    cudaError_t e = clear_error_and_counters(g, ws, s);
     if (e != cudaSuccess) return e;
     if (g.N == 0)  // no Gaussians: every tile list empty at 0
         return cudaMemsetAsync(ws.offs, 0, sizeof(int) * (size_t)g.B * (g.T + 1), s);

@@ -47,6 +47,8 @@ struct Geom {
     int out_vec2;       // 1 if the output image allows 8-byte 2-pixel stores
     int out_vec4;       // 1 if the output image allows 16-byte 4-pixel stores
     int img_dtype;      // storage of image / dL/dI: PDR_F32, PDR_F16 or PDR_BF16
+    int bwd_threads;    // threads per backward block
+    int bwd_rcap;       // home records a backward block stages at most (>= its threads)
 };
 
 constexpr int kBinChunk = 1024;        // Gaussians per binning block (large frames)
@@ -64,6 +66,7 @@ constexpr int kClusterMaxBlocks = 4 * 148;   // ... while the launch has at most
 // weight is w = 2^{-(uhat_1^2 + uhat_2^2)} = exp(-q / 2).
 struct Workspace {
     int *err;       // device error word
+    int *done;      // [B] per-frame block counters of the tile scan (zero between launches)
     float4 *gr;     // [B*N][2]
     int *hist;      // [B][nchunks][T]: chunk counts, then prefix over chunks
     int *offs;      // [B][T + 1]: absolute list start of every tile, frame end
@@ -218,7 +221,8 @@ size_t bin_frame_smem(const Geom &g);
 size_t bin_count_smem(const Geom &g);
 size_t bin_scatter_smem(const Geom &g);
 size_t bwd_smem(const Geom &g);
-size_t bwd_smem_nt(const Geom &g, int nt);
-int bwd_threads(const Geom &g);  // threads per block of the scalar backward
+// The backward kernel for these sizes: the pixel-pair kernel (C <= 4, k 13 or
+// 15) or the scalar one.
+bool bwd_uses_pairs(int C, int k);
 
 }  // namespace pdr

@@ -36,9 +36,6 @@ namespace pdr {
 namespace {
 
 constexpr int kGroup = 8;   // lanes per Gaussian
-constexpr int kPass = 256;  // list entries per pass = home records staged at most
-// List entries per thread per pass.
-template <int NT> struct Per { static constexpr int n = kPass / NT; };
 
 // Home record staged in shared memory (float4 units):
 //   [0] = (alpha_1, beta_1, K_1, alpha_2)   K_j = uhat_j at the window corner
@@ -58,40 +55,29 @@ __host__ __device__ __forceinline__ int staged_pitch(int RS, int k) {
     return RS + (((k - RS) % 8) + 8) % 8;
 }
 
-// One pass of a tile list: entry e0 + j * NT + tid (j < kPer) is held by
-// thread tid as raw[j] (binner entry with its home flag) when valid[j].
-// Returns each home entry's rank among the pass's home entries in list order
-// (-1 for others) and their total.  Called by the whole block; wcnt holds
-// kPass / 32 ints and may be reused after the caller's next barrier.
-template <int NT, int kPer = Per<NT>::n>
-__device__ __forceinline__ void home_ranks(const int (&raw)[kPer], const bool (&valid)[kPer],
-                                           int *wcnt, int (&pos)[kPer], int &total) {
+// One pass of a tile list: entry e0 + tid is held by thread tid as raw (the
+// binner's entry with its home flag) when valid.  Returns the entry's rank
+// among the pass's home entries in list order (-1 if it is not a home entry)
+// and their total.  Called by the whole block; consecutive passes alternate
+// between the two halves of wcnt ([2][NT / 32]), so that no thread can
+// overwrite counts another thread of the previous pass is still reading.
+template <int NT>
+__device__ __forceinline__ int home_rank(int raw, bool valid, int *wcnt, int &total) {
     constexpr int NW = NT / 32;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const unsigned lt = lanemask_lt();
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) {
-        const bool h = valid[j] && entry_home(raw[j]);
-        const unsigned bal = __ballot_sync(0xffffffffu, h);
-        pos[j] = h ? (int)__popc(bal & lt) : -1;
-        if (lane == 0) wcnt[j * NW + warp] = __popc(bal);
-    }
+    const bool h = valid && entry_home(raw);
+    const unsigned bal = __ballot_sync(0xffffffffu, h);
+    if (lane == 0) wcnt[warp] = __popc(bal);
     __syncthreads();
-    // List order is (j, warp, lane): add the counts of every earlier (j, warp).
-    int before[kPer];
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) before[j] = 0;
+    int before = 0;
     total = 0;
 #pragma unroll
-    for (int q = 0; q < kPer * NW; ++q) {
-        const int c = wcnt[q];
-#pragma unroll
-        for (int j = 0; j < kPer; ++j) before[j] += q < j * NW + warp ? c : 0;
+    for (int w = 0; w < NW; ++w) {
+        const int c = wcnt[w];
+        before += w < warp ? c : 0;
         total += c;
     }
-#pragma unroll
-    for (int j = 0; j < kPer; ++j)
-        if (pos[j] >= 0) pos[j] += before[j];
+    return h ? before + (int)__popc(bal & lanemask_lt()) : -1;
 }
 
 // The part of a home record that both kernels share: rows 0, 1 and the
@@ -201,9 +187,15 @@ __device__ __forceinline__ void load_gpix(const float *gh, int pix, float (&gv)[
 // ---------------------------------------------------------------------------
 // Scalar backward (any C, any k; common k compiled in).  Eight lanes stride
 // over a Gaussian's k*k window pixels (lane l takes pixels l, l + 8, ... in
-// row-major order, from a per-block offset table).  The staged rows have a
-// pitch congruent to k modulo 8, so the 8 pixels the lanes of a group read
-// together fall in 8 distinct 16-byte bank groups even across a row wrap.
+// row-major order, from a per-block offset table).  dL/dI is staged over
+// [X0 - 2r, X0 + 15 + 2r]^2, zero outside the core [X0 - r, X0 + 15 + r]^2
+// and outside the grid: the core holds the whole window of every home
+// Gaussian centred on the grid, and the outer ring is only read by home
+// Gaussians centred off the grid (a border tile's), at pixels that are
+// themselves off the grid, so every home Gaussian reads shared memory only.
+// The staged rows have a pitch congruent to k modulo 8, so the 8 pixels the
+// lanes of a group read together fall in 8 distinct 16-byte bank groups even
+// across a row wrap.
 // ---------------------------------------------------------------------------
 template <int C, int KT, int NT>
 __global__ void __launch_bounds__(NT, C > 4 ? 1 : 1024 / NT) k_bwd(const float *__restrict__ params,
@@ -217,23 +209,22 @@ __global__ void __launch_bounds__(NT, C > 4 ? 1 : 1024 / NT) k_bwd(const float *
     constexpr int NV = 5 + C;
     constexpr int RV = HRec<C>::RV;
     constexpr int NG = NT / kGroup;
-    constexpr int PASS = kPass;  // list entries per pass = staged record capacity
-    constexpr int kPer = Per<NT>::n;
     extern __shared__ float4 smem4[];
-    __shared__ int wcnt[kPass / 32];
+    __shared__ int wcnt[2][NT / 32];
     const int k = KT ? KT : g.k, r = (k - 1) / 2;
     const int RS = kTile + 4 * r;                 // staged region edge (pixels)
     const int RP = staged_pitch(RS, k);           // its row pitch
     const int kk = k * k;
     const int full = kk / kGroup, tail = kk - full * kGroup;  // compile-time when KT > 0
+    const int rcap = g.bwd_rcap;                  // home records staged at most
     float4 *table = smem4;                        // [(full + 1) * 8]: (ox, oy, offset, 0)
-    float4 *recs = table + (full + 1) * kGroup;   // [PASS][RV]
-    float *gh = reinterpret_cast<float *>(recs + PASS * RV);  // [RS*RP][GP]
+    float4 *recs = table + (full + 1) * kGroup;   // [rcap][RV]
+    float *gh = reinterpret_cast<float *>(recs + (size_t)rcap * RV);  // [RS*RP][GP]
     {
         // The launch must have provided this layout; otherwise report, touch nothing.
-        const unsigned need = (unsigned)(sizeof(float4) * ((full + 1) * kGroup + PASS * RV) +
+        const unsigned need = (unsigned)(sizeof(float4) * ((full + 1) * kGroup + rcap * RV) +
                                          sizeof(float) * RS * RP * GP);
-        if (dynamic_smem_bytes() < need) {
+        if (dynamic_smem_bytes() < need || rcap < NT) {
             if (threadIdx.x == 0) atomicOr(err, kErrSmemLayout);
             return;
         }
@@ -242,7 +233,7 @@ __global__ void __launch_bounds__(NT, C > 4 ? 1 : 1024 / NT) k_bwd(const float *
     const int b = blockIdx.x / g.T, t = blockIdx.x - b * g.T;
     const int ty = t / g.TX, tx = t - ty * g.TX;
     const int X0 = tx * kTile, Y0 = ty * kTile;
-    const int RX0 = X0 - 2 * r, RY0 = Y0 - 2 * r;  // region origin (grid coordinates)
+    const int RX0 = X0 - 2 * r, RY0 = Y0 - 2 * r;  // staged region origin (grid coordinates)
     const int tid = threadIdx.x;
     const int grp = tid / kGroup, lig = tid % kGroup;
     // Groups of one warp may run different numbers of Gaussians, so the
@@ -251,16 +242,10 @@ __global__ void __launch_bounds__(NT, C > 4 ? 1 : 1024 / NT) k_bwd(const float *
 
     int L0, L1;
     list_range(offs, g, b, t, err, L0, L1);
-    // The first pass's entries, requested before the staging loads so that
+    // The first pass's entry, requested before the staging loads so that
     // both are in flight together.
-    int raw[kPer];
-    bool valid[kPer];
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) {
-        const int e = L0 + j * NT + tid;
-        valid[j] = e < L1;
-        raw[j] = valid[j] ? ids[e] : 0;
-    }
+    bool valid = L0 + tid < L1;
+    int raw = valid ? ids[L0 + tid] : 0;
 
     zero_missing(gr, g, b, t, dparams);
 
@@ -271,9 +256,7 @@ __global__ void __launch_bounds__(NT, C > 4 ? 1 : 1024 / NT) k_bwd(const float *
         const int ox = p % k, oy = p / k;
         table[j] = make_float4((float)ox, (float)oy, __int_as_float(oy * RP + ox), 0.0f);
     }
-    // dL/dI of the core [X0 - r, X0 + 15 + r]^2 (zero outside the grid); the
-    // outer ring is only ever read by Gaussians centred off the grid, at
-    // pixels that are themselves off the grid, so it is all zeros.
+    // dL/dI of the core (zero outside it and outside the grid).
     constexpr int kStageU = 4;  // pixels per thread with their loads in flight together
     for (int p0 = 0; p0 < RS * RS; p0 += kStageU * NT) {
         float v[kStageU][GP];
@@ -307,44 +290,14 @@ __global__ void __launch_bounds__(NT, C > 4 ? 1 : 1024 / NT) k_bwd(const float *
         }
     }
 
-    for (int e0 = L0; e0 < L1; e0 += PASS) {
-        if (e0 != L0) {
-#pragma unroll
-            for (int j = 0; j < kPer; ++j) {
-                const int e = e0 + j * NT + tid;
-                valid[j] = e < L1;
-                raw[j] = valid[j] ? ids[e] : 0;
-            }
-        }
-        int pos[kPer], nh;
-        home_ranks<NT>(raw, valid, wcnt, pos, nh);
-#pragma unroll
-        for (int j = 0; j < kPer; ++j) {
-            if (pos[j] < 0) continue;
-            float4 R[RV];
-            const int id = entry_id(raw[j]);
-            if (id >= g.N) {  // never for consistent bins
-                atomicOr(err, kErrBadId);
-                R[1] = make_float4(0.0f, 0.0f, 0.0f, __int_as_float(-1));
-                recs[pos[j] * RV + 1] = R[1];
-                continue;
-            }
-            int cx, cy;
-            home_record_common<C>(params, gr, g, b, id, cx, cy, R);
-            const int gboff = (((cy - r) - RY0) * RP + ((cx - r) - RX0)) * GP;
-            R[2] = make_float4(__int_as_float(gboff), 0.0f, 0.0f, 0.0f);
-#pragma unroll
-            for (int v = 0; v < RV; ++v) recs[pos[j] * RV + v] = R[v];
-        }
-        __syncthreads();  // records visible; wcnt free again
-
-        for (int h = grp; h < nh; h += NG) {
+    // The staged home Gaussians recs[0 .. n), one per group at a time.
+    auto process = [&](int n) {
+        for (int h = grp; h < n; h += NG) {
             const float4 *R = recs + h * RV;
-            const float4 r0 = R[0], r1 = R[1];
+            const float4 r0 = R[0], r1 = R[1], r2 = R[2];
             const int id = __float_as_int(r1.w);
             if (id < 0) continue;
             const float a1 = r0.x, b1 = r0.y, K1 = r0.z, a2 = r0.w, b2 = r1.x, K2 = r1.y;
-            const float *gb = gh + __float_as_int(R[2].x);
             float amp[4 * (RV - 3)];
 #pragma unroll
             for (int v = 0; v < RV - 3; ++v) {
@@ -355,12 +308,9 @@ __global__ void __launch_bounds__(NT, C > 4 ? 1 : 1024 / NT) k_bwd(const float *
 #pragma unroll
             for (int j = 0; j < NV; ++j) acc[j] = 0.0f;
 
-            auto eval = [&](int j) {
-                const float4 tb = table[j * kGroup + lig];
-                float gv[C];
-                load_gpix<C>(gb, __float_as_int(tb.z), gv);
-                const float u1 = fmaf(a1, tb.x, fmaf(b1, tb.y, K1));
-                const float u2 = fmaf(a2, tb.x, fmaf(b2, tb.y, K2));
+            auto pixel = [&](float ox, float oy, const float (&gv)[C]) {
+                const float u1 = fmaf(a1, ox, fmaf(b1, oy, K1));
+                const float u2 = fmaf(a2, ox, fmaf(b2, oy, K2));
                 const float w = ex2(fmaf(-u1, u1, -u2 * u2));
                 float G = gv[0] * amp[0];
 #pragma unroll
@@ -374,6 +324,13 @@ __global__ void __launch_bounds__(NT, C > 4 ? 1 : 1024 / NT) k_bwd(const float *
                 acc[2] = fmaf(vu1, u1, acc[2]);
                 acc[3] = fmaf(vu1, u2, acc[3]);
                 acc[4] = fmaf(vu2, u2, acc[4]);
+            };
+            const float *gb = gh + __float_as_int(r2.x);
+            auto eval = [&](int j) {
+                const float4 tb = table[j * kGroup + lig];
+                float gv[C];
+                load_gpix<C>(gb, __float_as_int(tb.z), gv);
+                pixel(tb.x, tb.y, gv);
             };
             if constexpr (KT > 0) {
 #pragma unroll 8
@@ -398,8 +355,43 @@ __global__ void __launch_bounds__(NT, C > 4 ? 1 : 1024 / NT) k_bwd(const float *
             for (int j = 0; j < Extra<C>::n; ++j) extra[j] = 8 + j < NV ? acc[8 + j < NV ? 8 + j : 0] : 0.0f;
             group_write<C>(v, extra, gmask, lig, dparams + ((size_t)b * g.N + id) * g.P);
         }
-        __syncthreads();  // records consumed before the next pass overwrites them
+    };
+
+    // Passes of NT list entries: the home entries' records are gathered into
+    // recs until the next pass could overflow it, then processed.
+    int nh = 0, pass = 0;
+    for (int e0 = L0; e0 < L1; e0 += NT, ++pass) {
+        if (e0 != L0) {
+            valid = e0 + tid < L1;
+            raw = valid ? ids[e0 + tid] : 0;
+        }
+        int tot;
+        const int pos = home_rank<NT>(raw, valid, wcnt[pass & 1], tot);
+        if (nh + tot > rcap) {  // block-uniform
+            process(nh);
+            __syncthreads();  // records consumed before they are overwritten
+            nh = 0;
+        }
+        if (pos >= 0) {
+            float4 R[RV];
+            const int id = entry_id(raw);
+            if (id >= g.N) {  // never for consistent bins
+                atomicOr(err, kErrBadId);
+                recs[(nh + pos) * RV + 1] = make_float4(0.0f, 0.0f, 0.0f, __int_as_float(-1));
+            } else {
+                int cx, cy;
+                home_record_common<C>(params, gr, g, b, id, cx, cy, R);
+                const int wx0 = cx - r, wy0 = cy - r;  // inside the staged region
+                R[2] = make_float4(__int_as_float(((wy0 - RY0) * RP + (wx0 - RX0)) * GP), 0.0f,
+                                   0.0f, 0.0f);
+#pragma unroll
+                for (int v = 0; v < RV; ++v) recs[(nh + pos) * RV + v] = R[v];
+            }
+        }
+        nh += tot;
     }
+    __syncthreads();  // the last pass's records (and the staging) visible
+    process(nh);
 }
 
 // ---------------------------------------------------------------------------
@@ -445,14 +437,14 @@ struct PairShape {
     static constexpr int PLANE = ROWS * PITCH;               // elements per (parity, plane)
     static constexpr int NIT = ROWS * PAIRS;                 // staging items
     static constexpr int RV = HRec<C>::RV;
-    static constexpr int PASS = kPass;
     static constexpr size_t HALO4 = sizeof(float4) * 2 * NP4 * PLANE;
     static constexpr size_t HALO2 = sizeof(float2) * 2 * NP2 * PLANE;
-    static constexpr size_t SMEM = HALO4 + HALO2 + sizeof(float4) * RV * PASS;
+    // Dynamic shared memory for a record capacity of rcap home Gaussians.
+    __host__ __device__ static constexpr size_t smem(int rcap) { return HALO4 + HALO2 + sizeof(float4) * RV * rcap; }
 };
 
 template <int C, int K, int NT>
-__global__ void __launch_bounds__(NT, 640 / NT) k_bwd_pairs(const float *__restrict__ params,
+__global__ void __launch_bounds__(NT, 896 / NT) k_bwd_pairs(const float *__restrict__ params,
                                                   const void *__restrict__ gimg, Geom g,
                                                   const float4 *__restrict__ gr,
                                                   const int *__restrict__ offs,
@@ -461,17 +453,17 @@ __global__ void __launch_bounds__(NT, 640 / NT) k_bwd_pairs(const float *__restr
                                                   int *__restrict__ err) {
     using S = PairShape<C, K, NT>;
     constexpr int R = S::R, NPW = S::NPW, NS = S::NS, NP4 = S::NP4, NP2 = S::NP2;
-    constexpr int RV = S::RV, NG = NT / kGroup, PASS = S::PASS;
-    constexpr int kPer = Per<NT>::n;
+    constexpr int RV = S::RV, NG = NT / kGroup;
     constexpr int NCH = 2 * NP4 + NP2;  // channels staged per pixel (C, rounded to the planes)
     extern __shared__ float4 smem4[];
-    __shared__ int wcnt[kPass / 32];
+    __shared__ int wcnt[2][NT / 32];
+    const int rcap = g.bwd_rcap;  // home records staged at most
     float4 *halo4 = smem4;                                             // [parity][NP4][ROWS][PITCH]
     float2 *halo2 = reinterpret_cast<float2 *>(smem4 + 2 * NP4 * S::PLANE);  // [parity][ROWS][PITCH]
-    float4 *recs = smem4 + (S::HALO4 + S::HALO2) / sizeof(float4);    // [PASS][RV]
+    float4 *recs = smem4 + (S::HALO4 + S::HALO2) / sizeof(float4);    // [rcap][RV]
     static_assert(S::HALO2 % sizeof(float4) == 0, "record area must stay 16-byte aligned");
-    if (dynamic_smem_bytes() < (unsigned)S::SMEM || g.k != K) {  // launch/layout mismatch
-        if (threadIdx.x == 0) atomicOr(err, kErrSmemLayout);
+    if (dynamic_smem_bytes() < (unsigned)S::smem(rcap) || g.k != K || rcap < NT) {
+        if (threadIdx.x == 0) atomicOr(err, kErrSmemLayout);  // launch/layout mismatch
         return;
     }
 
@@ -485,14 +477,10 @@ __global__ void __launch_bounds__(NT, 640 / NT) k_bwd_pairs(const float *__restr
 
     int L0, L1;
     list_range(offs, g, b, t, err, L0, L1);
-    int raw[kPer];
-    bool valid[kPer];
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) {
-        const int e = L0 + j * NT + tid;
-        valid[j] = e < L1;
-        raw[j] = valid[j] ? ids[e] : 0;
-    }
+    // The first pass's entry, requested before the staging loads so that
+    // both are in flight together.
+    bool valid = L0 + tid < L1;
+    int raw = valid ? ids[L0 + tid] : 0;
 
     // Stage dL/dI over [X0 - r, X0 + 15 + r]^2 (zero outside the grid; the
     // column after it, read only as the masked pixel of a last pair, is zero
@@ -541,52 +529,21 @@ __global__ void __launch_bounds__(NT, 640 / NT) k_bwd_pairs(const float *__restr
 
     // This lane's pair column and first row (independent of the Gaussian),
     // with the mask of the pair's second pixel (last pair of a row).
-    const bool lane_on = lig < S::LANES;
-    const int pc = lig % NPW, r0 = lig / NPW;
+    // With one row per lane step (RPS == 1) every active lane starts on row 0
+    // and its last row is the window's last; with all 8 lanes active (k = 15)
+    // no lane idles: both tests are then compile-time constants.
+    constexpr bool kAllOn = S::LANES == kGroup;
+    const bool lane_on = kAllOn || lig < S::LANES;
+    const int pc = lig % NPW, r0 = S::RPS == 1 ? 0 : lig / NPW;
     const float2 sfx = make_float2((float)(2 * pc), (float)(2 * pc + 1));
     const float2 sfy = f2dup((float)r0);
     const float smask = pc == NPW - 1 ? __int_as_float(0x7f800000) : 0.0f;  // +inf: 2^-inf = 0
     const int soff = r0 * S::PITCH + pc;
-    const bool last_ok = r0 + (NS - 1) * S::RPS < K;  // the lane's last row lies in the window
+    const bool last_ok = S::RPS == 1 || r0 + (NS - 1) * S::RPS < K;  // the lane's last row lies in the window
 
-    for (int e0 = L0; e0 < L1; e0 += PASS) {
-        if (e0 != L0) {
-#pragma unroll
-            for (int j = 0; j < kPer; ++j) {
-                const int e = e0 + j * NT + tid;
-                valid[j] = e < L1;
-                raw[j] = valid[j] ? ids[e] : 0;
-            }
-        }
-        int pos[kPer], nh;
-        home_ranks<NT>(raw, valid, wcnt, pos, nh);
-#pragma unroll
-        for (int j = 0; j < kPer; ++j) {
-            if (pos[j] < 0) continue;
-            float4 Rr[RV];
-            const int id = entry_id(raw[j]);
-            if (id >= g.N) {  // never for consistent bins
-                atomicOr(err, kErrBadId);
-                recs[pos[j] * RV + 1] = make_float4(0.0f, 0.0f, 0.0f, __int_as_float(-1));
-                continue;
-            }
-            int cx, cy;
-            home_record_common<C>(params, gr, g, b, id, cx, cy, Rr);
-            const int wx0 = cx - R, wy0 = cy - R;
-            const bool ongrid = cx >= 0 && cx < g.W && cy >= 0 && cy < g.H;
-            const int lx = wx0 - RX0;  // in [0, 15] on the grid
-            const int el = (wy0 - RY0) * S::PITCH + (lx >> 1);
-            Rr[2] = ongrid ? make_float4(__int_as_float((lx & 1) * NP4 * S::PLANE + el),
-                                         __int_as_float((lx & 1) * S::PLANE + el), 0.0f,
-                                         __int_as_float(1))
-                           : make_float4(__int_as_float(wx0), __int_as_float(wy0), 0.0f,
-                                         __int_as_float(0));
-#pragma unroll
-            for (int v = 0; v < RV; ++v) recs[pos[j] * RV + v] = Rr[v];
-        }
-        __syncthreads();  // records (and, in the first pass, the halo) visible
-
-        for (int h = grp; h < nh; h += NG) {
+    // The staged home Gaussians recs[0 .. n), one per group at a time.
+    auto process = [&](int n) {
+        for (int h = grp; h < n; h += NG) {
             const float4 *Rh = recs + h * RV;
             const float4 q0 = Rh[0], q1 = Rh[1], q2 = Rh[2];
             const int id = __float_as_int(q1.w);
@@ -695,15 +652,55 @@ __global__ void __launch_bounds__(NT, 640 / NT) k_bwd_pairs(const float *__restr
             float extra[Extra<C>::n] = {C > 3 ? DA[C > 3 ? 3 : 0].x + DA[C > 3 ? 3 : 0].y : 0.0f};
             group_write<C>(v, extra, gmask, lig, dparams + ((size_t)b * g.N + id) * g.P);
         }
-        __syncthreads();  // records consumed before the next pass overwrites them
+    };
+
+    // Passes of NT list entries: the home entries' records are gathered into
+    // recs until the next pass could overflow it, then processed.
+    int nh = 0, pass = 0;
+    for (int e0 = L0; e0 < L1; e0 += NT, ++pass) {
+        if (e0 != L0) {
+            valid = e0 + tid < L1;
+            raw = valid ? ids[e0 + tid] : 0;
+        }
+        int tot;
+        const int pos = home_rank<NT>(raw, valid, wcnt[pass & 1], tot);
+        if (nh + tot > rcap) {  // block-uniform
+            process(nh);
+            __syncthreads();  // records consumed before they are overwritten
+            nh = 0;
+        }
+        if (pos >= 0) {
+            float4 Rr[RV];
+            const int id = entry_id(raw);
+            if (id >= g.N) {  // never for consistent bins
+                atomicOr(err, kErrBadId);
+                recs[(nh + pos) * RV + 1] = make_float4(0.0f, 0.0f, 0.0f, __int_as_float(-1));
+            } else {
+                int cx, cy;
+                home_record_common<C>(params, gr, g, b, id, cx, cy, Rr);
+                const int wx0 = cx - R, wy0 = cy - R;
+                const bool ongrid = cx >= 0 && cx < g.W && cy >= 0 && cy < g.H;
+                const int lx = wx0 - RX0;  // in [0, 15] on the grid
+                const int el = (wy0 - RY0) * S::PITCH + (lx >> 1);
+                Rr[2] = ongrid ? make_float4(__int_as_float((lx & 1) * NP4 * S::PLANE + el),
+                                             __int_as_float((lx & 1) * S::PLANE + el), 0.0f,
+                                             __int_as_float(1))
+                               : make_float4(__int_as_float(wx0), __int_as_float(wy0), 0.0f,
+                                             __int_as_float(0));
+#pragma unroll
+                for (int v = 0; v < RV; ++v) recs[(nh + pos) * RV + v] = Rr[v];
+            }
+        }
+        nh += tot;
     }
+    __syncthreads();  // the last pass's records (and the staging) visible
+    process(nh);
 }
 
 template <int C, int K, int NT>
 cudaError_t launch_bwd_pairs(const float *params, const void *grad_image, const Geom &g,
                              const Workspace &ws, float *grad_params, cudaStream_t s) {
-    constexpr size_t smem = PairShape<C, K, NT>::SMEM;
-    static_assert(smem <= 200 * 1024, "staged dL/dI does not fit");
+    const size_t smem = PairShape<C, K, NT>::smem(g.bwd_rcap);
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(k_bwd_pairs<C, K, NT>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -717,7 +714,7 @@ cudaError_t launch_bwd_pairs(const float *params, const void *grad_image, const 
 template <int C, int KT, int NT>
 cudaError_t launch_bwd_ck(const float *params, const void *grad_image, const Geom &g,
                           const Workspace &ws, float *grad_params, cudaStream_t s) {
-    const size_t smem = bwd_smem_nt(g, NT);
+    const size_t smem = bwd_smem(g);
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(k_bwd<C, KT, NT>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -731,8 +728,8 @@ cudaError_t launch_bwd_ck(const float *params, const void *grad_image, const Geo
 template <int C, int KT>
 cudaError_t launch_bwd_scalar(const float *params, const void *grad_image, const Geom &g,
                               const Workspace &ws, float *grad_params, cudaStream_t s) {
-    return bwd_threads(g) == 128 ? launch_bwd_ck<C, KT, 128>(params, grad_image, g, ws, grad_params, s)
-                                 : launch_bwd_ck<C, KT, 256>(params, grad_image, g, ws, grad_params, s);
+    return g.bwd_threads == 128 ? launch_bwd_ck<C, KT, 128>(params, grad_image, g, ws, grad_params, s)
+                                : launch_bwd_ck<C, KT, 256>(params, grad_image, g, ws, grad_params, s);
 }
 
 template <int C>
@@ -756,27 +753,18 @@ cudaError_t launch_bwd_c(const float *params, const void *grad_image, const Geom
 
 }  // namespace
 
-// Threads per block of the scalar backward: 128 when a tile holds few home
-// Gaussians on average (the last round of 8-lane groups is then short),
-// 256 otherwise.
-int bwd_threads(const Geom &g) {
-    const long long per_tile = ((long long)g.N + g.T - 1) / g.T;
-    return per_tile <= 128 ? 128 : 256;
-}
+bool bwd_uses_pairs(int C, int k) { return C <= 4 && (k == 13 || k == 15); }
 
-size_t bwd_smem_nt(const Geom &g, int nt) {
+size_t bwd_smem(const Geom &g) {
     const int kk = g.k * g.k;
     const int full = kk / kGroup;
     const int RS = kTile + 4 * g.r;
     const int RP = staged_pitch(RS, g.k);
     const int GP = g.C <= 1 ? 1 : g.C <= 2 ? 2 : g.C <= 4 ? 4 : 8;
     const int RV = 3 + (g.C + 3) / 4;
-    (void)nt;  // the record area holds kPass records whatever the block size
-    return sizeof(float4) * ((size_t)(full + 1) * kGroup + (size_t)kPass * RV) +
+    return sizeof(float4) * ((size_t)(full + 1) * kGroup + (size_t)g.bwd_rcap * RV) +
            sizeof(float) * (size_t)RS * RP * GP;
 }
-
-size_t bwd_smem(const Geom &g) { return bwd_smem_nt(g, bwd_threads(g)); }
 
 cudaError_t launch_bwd(const float *params, const void *grad_image, const Geom &g,
                        const Workspace &ws, float *grad_params, cudaStream_t s) {

@@ -64,23 +64,7 @@ struct FwdSmem {
     unsigned win[NB];  // window as column bits | row bits << 16 (tile pixels)
     unsigned sub[16][NB];
     int subn[16];
-    // pen[m].j = 0 if bit j of m is set, else +inf: added to the quadratic
-    // form of a lane's pixel j, it turns the weight of a pixel outside the
-    // window into 2^-inf = 0 without a branch or a predicate per pixel.
-    float4 pen[16];
 };
-
-__device__ __forceinline__ float2 f2fma(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
-
-template <int C, int NB>
-__device__ __forceinline__ void init_pen(FwdSmem<C, NB> &S) {
-    if (threadIdx.x < 16) {
-        const float inf = __int_as_float(0x7f800000);
-        const unsigned m = threadIdx.x;
-        S.pen[m] = make_float4(m & 1u ? 0.0f : inf, m & 2u ? 0.0f : inf, m & 4u ? 0.0f : inf,
-                               m & 8u ? 0.0f : inf);
-    }
-}
 
 // Render the entries list[0 .. L) (frame-local ids, ascending) of the tile at
 // (X0, Y0) of frame b into acc.  Called by the whole block.
@@ -89,7 +73,7 @@ __device__ __forceinline__ void init_pen(FwdSmem<C, NB> &S) {
 template <int C, int PL, int NB, typename Fetch>
 __device__ __forceinline__ void render_list(const Geom &g, Fetch fetch, const int *list,
                                             int L, int X0, int Y0, int *err,
-                                            FwdSmem<C, NB> &S, float2 (&acc)[PL / 2][C]) {
+                                            FwdSmem<C, NB> &S, float (&acc)[PL][C]) {
     using LY = FwdLayout<PL>;
     constexpr int RV = FwdRec<C>::kVec;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -172,10 +156,6 @@ __device__ __forceinline__ void render_list(const Geom &g, Fetch fetch, const in
         __syncthreads();
         const int ns = S.subn[grp];
         const unsigned *sl = S.sub[grp];
-        // Pixel pairs (x, x + 1) of the lane's run with the packed f32x2
-        // arithmetic of sm_100: one instruction per pair for each step of the
-        // quadratic form and each channel's accumulation.  A pixel outside the
-        // window gets +inf added to its quadratic form (weight exactly 0).
         for (int s = 0; s < ns; ++s) {
             const unsigned pk = sl[s];
             const float4 *r4 = reinterpret_cast<const float4 *>(
@@ -186,23 +166,20 @@ __device__ __forceinline__ void render_list(const Geom &g, Fetch fetch, const in
                 const float4 q = r4[v];
                 rr[4 * v] = q.x; rr[4 * v + 1] = q.y; rr[4 * v + 2] = q.z; rr[4 * v + 3] = q.w;
             }
-            const float4 P = S.pen[(pk >> bitshift) & 0xfu];
-            const float a1 = rr[0], a2 = rr[3];
-            const float u1 = fmaf(a1, fx, fmaf(rr[1], fy, rr[2]));
-            const float u2 = fmaf(a2, fx, fmaf(rr[4], fy, rr[5]));
-            float2 U1 = make_float2(u1, u1 + a1), U2 = make_float2(u2, u2 + a2);
+            const unsigned bits = pk >> bitshift;
+            float u1 = fmaf(rr[0], fx, fmaf(rr[1], fy, rr[2]));
+            float u2 = fmaf(rr[3], fx, fmaf(rr[4], fy, rr[5]));
 #pragma unroll
-            for (int h = 0; h < PL / 2; ++h) {
-                if (h) {
-                    const float d1 = a1 + a1, d2 = a2 + a2;
-                    U1 = make_float2(U1.x + d1, U1.y + d1);
-                    U2 = make_float2(U2.x + d2, U2.y + d2);
+            for (int j = 0; j < PL; ++j) {
+                if (j) {
+                    u1 += rr[0];
+                    u2 += rr[3];
                 }
-                const float2 pen = h ? make_float2(P.z, P.w) : make_float2(P.x, P.y);
-                const float2 q = f2fma(U1, U1, f2fma(U2, U2, pen));
-                const float2 w = make_float2(ex2(-q.x), ex2(-q.y));
+                const float w = ex2(fmaf(-u1, u1, -u2 * u2));
+                if (bits & (1u << j)) {
 #pragma unroll
-                for (int c = 0; c < C; ++c) acc[h][c] = f2fma(make_float2(rr[6 + c], rr[6 + c]), w, acc[h][c]);
+                    for (int c = 0; c < C; ++c) acc[j][c] = fmaf(rr[6 + c], w, acc[j][c]);
+                }
             }
         }
     }
@@ -210,15 +187,7 @@ __device__ __forceinline__ void render_list(const Geom &g, Fetch fetch, const in
 
 template <int C, int PL>
 __device__ __forceinline__ void store_tile(const Geom &g, int b, int X0, int Y0,
-                                           void *__restrict__ image_, const float2 (&acc2)[PL / 2][C]) {
-    float acc[PL][C];
-#pragma unroll
-    for (int h = 0; h < PL / 2; ++h)
-#pragma unroll
-        for (int c = 0; c < C; ++c) {
-            acc[2 * h][c] = acc2[h][c].x;
-            acc[2 * h + 1][c] = acc2[h][c].y;
-        }
+                                           void *__restrict__ image_, const float (&acc)[PL][C]) {
     using LY = FwdLayout<PL>;
     const int tid = threadIdx.x;
     const int grp = tid / LY::kLanes, lig = tid % LY::kLanes;
@@ -265,12 +234,11 @@ __global__ void __launch_bounds__(FwdLayout<PL>::kThreads) k_fwd(const float *__
     const int b = blockIdx.x / g.T, t = blockIdx.x - b * g.T;
     const int ty = t / g.TX, tx = t - ty * g.TX;
     const int X0 = tx * kTile, Y0 = ty * kTile;
-    float2 acc[PL / 2][C];
+    float acc[PL][C];
 #pragma unroll
-    for (int j = 0; j < PL / 2; ++j)
+    for (int j = 0; j < PL; ++j)
 #pragma unroll
-        for (int c = 0; c < C; ++c) acc[j][c] = make_float2(0.0f, 0.0f);
-    init_pen(S);
+        for (int c = 0; c < C; ++c) acc[j][c] = 0.0f;
     int L0, L1;
     list_range(offs, g, b, t, err, L0, L1);
     auto fetch = [&](int i, float4 &A, float4 &Q, float (&amp)[C]) {
@@ -311,7 +279,6 @@ __global__ void __launch_bounds__(FwdLayout<PL>::kThreads) k_fwd_cluster(
     const unsigned lt = lanemask_lt();
     if (tid < kClusterTiles) cnt[tid] = 0;
     if (tid < NW * kClusterTiles) masks[tid / kClusterTiles][tid % kClusterTiles] = 0u;
-    init_pen(S);
     __syncthreads();
 
     // 1. records and per-tile counts of this block's chunk
@@ -417,11 +384,11 @@ __global__ void __launch_bounds__(FwdLayout<PL>::kThreads) k_fwd_cluster(
     // 4. render this tile from its own list
     const int ty = q / g.TX, tx = q - ty * g.TX;
     const int X0 = tx * kTile, Y0 = ty * kTile;
-    float2 acc[PL / 2][C];
+    float acc[PL][C];
 #pragma unroll
-    for (int j = 0; j < PL / 2; ++j)
+    for (int j = 0; j < PL; ++j)
 #pragma unroll
-        for (int c = 0; c < C; ++c) acc[j][c] = make_float2(0.0f, 0.0f);
+        for (int c = 0; c < C; ++c) acc[j][c] = 0.0f;
     const int L = tstart[q + 1] - tstart[q];
     const int *src = L <= kClusterListCap ? list : ids + frame0 + tstart[q];
     if (onchip) {
