@@ -41,14 +41,23 @@ pdr_status make_geom(int B, int N, int C, int H, int W, int k, Geom *g) {
     g->P = 5 + C;
     g->m = (int)m;
     g->cap = (int)cap;
-    g->nchunks = (N + kBinChunk - 1) / kBinChunk;
+    // Chunks of 1024 Gaussians, halved (down to 256) while the launch would
+    // have fewer than two binning blocks per SM.
+    {
+        int ch = kBinChunk;
+        while (ch > kBinChunkMin && (long long)B * ((N + ch - 1) / ch) < 2 * 148) ch >>= 1;
+        g->chunk = ch;
+        g->nchunks = (N + ch - 1) / ch;
+    }
     int nw = kScatterWarps;  // scatter block: as many warps as the per-warp tile tables allow
     while (nw > 1 && (size_t)T * (6 * nw + 4) + 16 > kScatterSmemLimit) nw >>= 1;
     if ((size_t)T * (6 * nw + 4) + 16 > kScatterSmemLimit) return PDR_ERR_TOO_LARGE;
     g->scatter_warps = nw;
     // Small frames: one binning block per frame (its shared-memory tables
     // hold [2 + 2 * warps] x T ints).
-    g->frame_block = T <= kFrameBlockMaxT && N <= kFrameBlockMaxN;
+    // (only when the frames alone give at least one block per SM; otherwise
+    // the chunked kernels spread the work over more blocks)
+    g->frame_block = T <= kFrameBlockMaxT && N <= kFrameBlockMaxN && B >= 148;
     int ft = ((N + 31) / 32) * 32;
     if (ft > 1024) ft = 1024;
     if (ft < 32) ft = 32;

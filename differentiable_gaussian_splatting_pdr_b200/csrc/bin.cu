@@ -5,7 +5,7 @@
 // ascending id is the one the oracle also uses.  Three kernels on the
 // caller's stream, no float atomics, no host synchronisation:
 //
-//   k_count   one block per (frame, chunk of kBinChunk Gaussians): the
+//   k_count   one block per (frame, chunk of 256 .. 1024 Gaussians): the
 //             per-Gaussian record (window centre, rotated and scaled axes)
 //             and the chunk's per-tile counts (integer shared-memory atomics
 //             count only; they never decide a position);
@@ -39,8 +39,8 @@ __global__ void __launch_bounds__(kCountThreads) k_count(const float *__restrict
     const int b = blockIdx.y, c = blockIdx.x;
     for (int t = threadIdx.x; t < g.T; t += blockDim.x) hs[t] = 0;
     __syncthreads();
-    const int i0 = c * kBinChunk, i1 = min(i0 + kBinChunk, g.N);
-    constexpr int U = kBinChunk / kCountThreads;  // Gaussians per thread, all in flight
+    const int i0 = c * g.chunk, i1 = min(i0 + g.chunk, g.N);
+    constexpr int U = kBinChunk / kCountThreads;  // Gaussians per thread at most, all in flight
     float4 A[U], Q[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
@@ -160,7 +160,7 @@ __global__ void __launch_bounds__(1024) k_scan_tiles(Geom g, int *__restrict__ h
 }
 
 // Stable scatter of one chunk: warp w of the block owns the contiguous slab
-// [c * kBinChunk + w * S, + S) of the chunk (S = kBinChunk / warps), so list
+// [c * chunk + w * S, + S) of the chunk (S = chunk / warps), so list
 // order = (warp, sub-round of 32, lane) = ascending id.  Each lane loads the
 // window centres of all its Gaussians first (every load in flight at once)
 // and keeps them in registers for both passes:
@@ -294,8 +294,8 @@ __global__ void k_scatter(Geom g, const float4 *__restrict__ gr, const int *__re
     const int *hsrc = hist + ((size_t)b * g.nchunks + c) * T;
     const int *osrc = offs + (size_t)b * (T + 1);
     for (int t = threadIdx.x; t < T; t += blockDim.x) tbase[t] = osrc[t] + hsrc[t];
-    const int S = kBinChunk / nw;
-    const int c0 = c * kBinChunk, c1 = min(c0 + kBinChunk, g.N);
+    const int S = g.chunk / nw;
+    const int c0 = c * g.chunk, c1 = min(c0 + g.chunk, g.N);
     const int i0 = min(c0 + warp * S, c1), i1 = min(i0 + S, c1);
     const bool resident = S <= 32 * kScatterSub;
     int cx[kScatterSub], cy[kScatterSub];

@@ -38,7 +38,8 @@ struct Geom {
     int P;              // parameters per Gaussian (5 + C)
     int m;              // most tiles a window can touch along one axis
     int cap;            // tile-list capacity per frame (N * m * m)
-    int nchunks;        // binning chunks per frame (kBinChunk Gaussians each)
+    int chunk;          // Gaussians per binning chunk (a power of two, <= kBinChunk)
+    int nchunks;        // binning chunks per frame
     int scatter_warps;  // warps per scatter block
     int frame_block;    // 1: small frames, one binning block per frame
     int frame_threads;  // threads of that block
@@ -51,7 +52,8 @@ struct Geom {
     int bwd_rcap;       // home records a backward block stages at most (>= its threads)
 };
 
-constexpr int kBinChunk = 1024;        // Gaussians per binning block (large frames)
+constexpr int kBinChunk = 1024;        // most Gaussians per binning chunk (large frames)
+constexpr int kBinChunkMin = 256;      // fewest (more chunks when there are few frames)
 constexpr int kFrameBlockMaxT = 256;   // small frames: at most this many tiles
 constexpr int kFrameBlockMaxN = 16384; // and at most this many Gaussians
 constexpr int kClusterTiles = 16;            // frames up to this many tiles: one cluster per frame

@@ -55,29 +55,93 @@ __host__ __device__ __forceinline__ int staged_pitch(int RS, int k) {
     return RS + (((k - RS) % 8) + 8) % 8;
 }
 
-// One pass of a tile list: entry e0 + tid is held by thread tid as raw (the
-// binner's entry with its home flag) when valid.  Returns the entry's rank
-// among the pass's home entries in list order (-1 if it is not a home entry)
-// and their total.  Called by the whole block; consecutive passes alternate
-// between the two halves of wcnt ([2][NT / 32]), so that no thread can
-// overwrite counts another thread of the previous pass is still reading.
-template <int NT>
-__device__ __forceinline__ int home_rank(int raw, bool valid, int *wcnt, int &total) {
+// List entries each thread holds per pass (a pass is KP * NT entries).
+constexpr int kPer = 2;
+
+// One pass of a tile list: entry e0 + j * NT + tid (j < KP) is held by thread
+// tid as raw[j] (the binner's entry with its home flag) when valid[j].
+// Returns each entry's rank among the pass's home entries in list order (-1
+// if it is not a home entry) and their total.  Called by the whole block;
+// wcnt holds KP * NT / 32 ints (consecutive passes alternate between two such
+// areas, so that no thread can overwrite counts another thread of the
+// previous pass is still reading).
+template <int NT, int KP>
+__device__ __forceinline__ void home_ranks(const int (&raw)[KP], const bool (&valid)[KP],
+                                           int *wcnt, int (&pos)[KP], int &total) {
     constexpr int NW = NT / 32;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const bool h = valid && entry_home(raw);
-    const unsigned bal = __ballot_sync(0xffffffffu, h);
-    if (lane == 0) wcnt[warp] = __popc(bal);
+    const unsigned lt = lanemask_lt();
+#pragma unroll
+    for (int j = 0; j < KP; ++j) {
+        const bool h = valid[j] && entry_home(raw[j]);
+        const unsigned bal = __ballot_sync(0xffffffffu, h);
+        pos[j] = h ? (int)__popc(bal & lt) : -1;
+        if (lane == 0) wcnt[j * NW + warp] = __popc(bal);
+    }
     __syncthreads();
-    int before = 0;
+    // List order is (j, warp, lane): add the counts of every earlier (j, warp).
+    int before[KP];
+#pragma unroll
+    for (int j = 0; j < KP; ++j) before[j] = 0;
     total = 0;
 #pragma unroll
-    for (int w = 0; w < NW; ++w) {
-        const int c = wcnt[w];
-        before += w < warp ? c : 0;
+    for (int q = 0; q < KP * NW; ++q) {
+        const int c = wcnt[q];
+#pragma unroll
+        for (int j = 0; j < KP; ++j) before[j] += q < j * NW + warp ? c : 0;
         total += c;
     }
-    return h ? before + (int)__popc(bal & lanemask_lt()) : -1;
+#pragma unroll
+    for (int j = 0; j < KP; ++j)
+        if (pos[j] >= 0) pos[j] += before[j];
+}
+
+// The ids of pass 0 of a tile list, requested by the caller before its
+// halo staging so that both are in flight together.
+template <int NT, int KP>
+__device__ __forceinline__ void load_pass(const int *__restrict__ ids, int e0, int L1,
+                                          int (&raw)[KP], bool (&valid)[KP]) {
+#pragma unroll
+    for (int j = 0; j < KP; ++j) {
+        const int e = e0 + j * NT + (int)threadIdx.x;
+        valid[j] = e < L1;
+        raw[j] = valid[j] ? ids[e] : 0;
+    }
+}
+
+// Walks the tile list [L0, L1) in passes of KP * NT entries (pass 0 already
+// in raw / valid), ranks each pass's home entries in list order and gathers
+// all their records in one round of loads (make(raw entry, slot) writes the
+// record of slot `slot`), calling process(n) on the staged records whenever
+// the record area (rcap) is full and once at the end.  Called by the whole
+// block; the staging done before it is visible to process.
+template <int NT, int KP, typename Make, typename Process>
+__device__ __forceinline__ void gather_homes(const int *__restrict__ ids, int L0, int L1,
+                                             int rcap, int *wcnt2, int (&raw)[KP],
+                                             bool (&valid)[KP], Make make, Process process) {
+    constexpr int W = KP * NT / 32;
+    int nh = 0, pass = 0;
+    for (int e0 = L0; e0 < L1; e0 += KP * NT, ++pass) {
+        if (e0 != L0) load_pass<NT, KP>(ids, e0, L1, raw, valid);
+        int pos[KP], tot;
+        home_ranks<NT, KP>(raw, valid, wcnt2 + (pass & 1) * W, pos, tot);
+        for (int done = 0; done < tot;) {  // block-uniform
+            if (nh == rcap) {
+                __syncthreads();  // the staged records visible
+                process(nh);
+                __syncthreads();  // records consumed before they are overwritten
+                nh = 0;
+            }
+            const int take = min(tot - done, rcap - nh);
+#pragma unroll
+            for (int j = 0; j < KP; ++j)
+                if (pos[j] >= done && pos[j] < done + take) make(raw[j], nh + pos[j] - done);
+            nh += take;
+            done += take;
+        }
+    }
+    __syncthreads();  // the last records (and the staging) visible
+    process(nh);
 }
 
 // The part of a home record that both kernels share: rows 0, 1 and the
@@ -210,7 +274,7 @@ __global__ void __launch_bounds__(NT, C > 4 ? 1 : 1024 / NT) k_bwd(const float *
     constexpr int RV = HRec<C>::RV;
     constexpr int NG = NT / kGroup;
     extern __shared__ float4 smem4[];
-    __shared__ int wcnt[2][NT / 32];
+    __shared__ int wcnt[2 * kPer * NT / 32];
     const int k = KT ? KT : g.k, r = (k - 1) / 2;
     const int RS = kTile + 4 * r;                 // staged region edge (pixels)
     const int RP = staged_pitch(RS, k);           // its row pitch
@@ -242,10 +306,11 @@ __global__ void __launch_bounds__(NT, C > 4 ? 1 : 1024 / NT) k_bwd(const float *
 
     int L0, L1;
     list_range(offs, g, b, t, err, L0, L1);
-    // The first pass's entry, requested before the staging loads so that
+    // The first pass's entries, requested before the staging loads so that
     // both are in flight together.
-    bool valid = L0 + tid < L1;
-    int raw = valid ? ids[L0 + tid] : 0;
+    int raw[kPer];
+    bool valid[kPer];
+    load_pass<NT, kPer>(ids, L0, L1, raw, valid);
 
     zero_missing(gr, g, b, t, dparams);
 
@@ -357,41 +422,22 @@ __global__ void __launch_bounds__(NT, C > 4 ? 1 : 1024 / NT) k_bwd(const float *
         }
     };
 
-    // Passes of NT list entries: the home entries' records are gathered into
-    // recs until the next pass could overflow it, then processed.
-    int nh = 0, pass = 0;
-    for (int e0 = L0; e0 < L1; e0 += NT, ++pass) {
-        if (e0 != L0) {
-            valid = e0 + tid < L1;
-            raw = valid ? ids[e0 + tid] : 0;
+    auto make = [&](int rawe, int slot) {
+        const int id = entry_id(rawe);
+        if (id >= g.N) {  // never for consistent bins
+            atomicOr(err, kErrBadId);
+            recs[slot * RV + 1] = make_float4(0.0f, 0.0f, 0.0f, __int_as_float(-1));
+            return;
         }
-        int tot;
-        const int pos = home_rank<NT>(raw, valid, wcnt[pass & 1], tot);
-        if (nh + tot > rcap) {  // block-uniform
-            process(nh);
-            __syncthreads();  // records consumed before they are overwritten
-            nh = 0;
-        }
-        if (pos >= 0) {
-            float4 R[RV];
-            const int id = entry_id(raw);
-            if (id >= g.N) {  // never for consistent bins
-                atomicOr(err, kErrBadId);
-                recs[(nh + pos) * RV + 1] = make_float4(0.0f, 0.0f, 0.0f, __int_as_float(-1));
-            } else {
-                int cx, cy;
-                home_record_common<C>(params, gr, g, b, id, cx, cy, R);
-                const int wx0 = cx - r, wy0 = cy - r;  // inside the staged region
-                R[2] = make_float4(__int_as_float(((wy0 - RY0) * RP + (wx0 - RX0)) * GP), 0.0f,
-                                   0.0f, 0.0f);
+        float4 R[RV];
+        int cx, cy;
+        home_record_common<C>(params, gr, g, b, id, cx, cy, R);
+        const int wx0 = cx - r, wy0 = cy - r;  // inside the staged region
+        R[2] = make_float4(__int_as_float(((wy0 - RY0) * RP + (wx0 - RX0)) * GP), 0.0f, 0.0f, 0.0f);
 #pragma unroll
-                for (int v = 0; v < RV; ++v) recs[(nh + pos) * RV + v] = R[v];
-            }
-        }
-        nh += tot;
-    }
-    __syncthreads();  // the last pass's records (and the staging) visible
-    process(nh);
+        for (int v = 0; v < RV; ++v) recs[slot * RV + v] = R[v];
+    };
+    gather_homes<NT, kPer>(ids, L0, L1, rcap, wcnt, raw, valid, make, process);
 }
 
 // ---------------------------------------------------------------------------
@@ -456,7 +502,7 @@ __global__ void __launch_bounds__(NT, 896 / NT) k_bwd_pairs(const float *__restr
     constexpr int RV = S::RV, NG = NT / kGroup;
     constexpr int NCH = 2 * NP4 + NP2;  // channels staged per pixel (C, rounded to the planes)
     extern __shared__ float4 smem4[];
-    __shared__ int wcnt[2][NT / 32];
+    __shared__ int wcnt[2 * kPer * NT / 32];
     const int rcap = g.bwd_rcap;  // home records staged at most
     float4 *halo4 = smem4;                                             // [parity][NP4][ROWS][PITCH]
     float2 *halo2 = reinterpret_cast<float2 *>(smem4 + 2 * NP4 * S::PLANE);  // [parity][ROWS][PITCH]
@@ -477,10 +523,11 @@ __global__ void __launch_bounds__(NT, 896 / NT) k_bwd_pairs(const float *__restr
 
     int L0, L1;
     list_range(offs, g, b, t, err, L0, L1);
-    // The first pass's entry, requested before the staging loads so that
+    // The first pass's entries, requested before the staging loads so that
     // both are in flight together.
-    bool valid = L0 + tid < L1;
-    int raw = valid ? ids[L0 + tid] : 0;
+    int raw[kPer];
+    bool valid[kPer];
+    load_pass<NT, kPer>(ids, L0, L1, raw, valid);
 
     // Stage dL/dI over [X0 - r, X0 + 15 + r]^2 (zero outside the grid; the
     // column after it, read only as the masked pixel of a last pair, is zero
@@ -654,47 +701,29 @@ __global__ void __launch_bounds__(NT, 896 / NT) k_bwd_pairs(const float *__restr
         }
     };
 
-    // Passes of NT list entries: the home entries' records are gathered into
-    // recs until the next pass could overflow it, then processed.
-    int nh = 0, pass = 0;
-    for (int e0 = L0; e0 < L1; e0 += NT, ++pass) {
-        if (e0 != L0) {
-            valid = e0 + tid < L1;
-            raw = valid ? ids[e0 + tid] : 0;
+    auto make = [&](int rawe, int slot) {
+        const int id = entry_id(rawe);
+        if (id >= g.N) {  // never for consistent bins
+            atomicOr(err, kErrBadId);
+            recs[slot * RV + 1] = make_float4(0.0f, 0.0f, 0.0f, __int_as_float(-1));
+            return;
         }
-        int tot;
-        const int pos = home_rank<NT>(raw, valid, wcnt[pass & 1], tot);
-        if (nh + tot > rcap) {  // block-uniform
-            process(nh);
-            __syncthreads();  // records consumed before they are overwritten
-            nh = 0;
-        }
-        if (pos >= 0) {
-            float4 Rr[RV];
-            const int id = entry_id(raw);
-            if (id >= g.N) {  // never for consistent bins
-                atomicOr(err, kErrBadId);
-                recs[(nh + pos) * RV + 1] = make_float4(0.0f, 0.0f, 0.0f, __int_as_float(-1));
-            } else {
-                int cx, cy;
-                home_record_common<C>(params, gr, g, b, id, cx, cy, Rr);
-                const int wx0 = cx - R, wy0 = cy - R;
-                const bool ongrid = cx >= 0 && cx < g.W && cy >= 0 && cy < g.H;
-                const int lx = wx0 - RX0;  // in [0, 15] on the grid
-                const int el = (wy0 - RY0) * S::PITCH + (lx >> 1);
-                Rr[2] = ongrid ? make_float4(__int_as_float((lx & 1) * NP4 * S::PLANE + el),
-                                             __int_as_float((lx & 1) * S::PLANE + el), 0.0f,
-                                             __int_as_float(1))
-                               : make_float4(__int_as_float(wx0), __int_as_float(wy0), 0.0f,
-                                             __int_as_float(0));
+        float4 Rr[RV];
+        int cx, cy;
+        home_record_common<C>(params, gr, g, b, id, cx, cy, Rr);
+        const int wx0 = cx - R, wy0 = cy - R;
+        const bool ongrid = cx >= 0 && cx < g.W && cy >= 0 && cy < g.H;
+        const int lx = wx0 - RX0;  // in [0, 15] on the grid
+        const int el = (wy0 - RY0) * S::PITCH + (lx >> 1);
+        Rr[2] = ongrid ? make_float4(__int_as_float((lx & 1) * NP4 * S::PLANE + el),
+                                     __int_as_float((lx & 1) * S::PLANE + el), 0.0f,
+                                     __int_as_float(1))
+                       : make_float4(__int_as_float(wx0), __int_as_float(wy0), 0.0f,
+                                     __int_as_float(0));
 #pragma unroll
-                for (int v = 0; v < RV; ++v) recs[(nh + pos) * RV + v] = Rr[v];
-            }
-        }
-        nh += tot;
-    }
-    __syncthreads();  // the last pass's records (and the staging) visible
-    process(nh);
+        for (int v = 0; v < RV; ++v) recs[slot * RV + v] = Rr[v];
+    };
+    gather_homes<NT, kPer>(ids, L0, L1, rcap, wcnt, raw, valid, make, process);
 }
 
 template <int C, int K, int NT>
@@ -728,8 +757,7 @@ cudaError_t launch_bwd_ck(const float *params, const void *grad_image, const Geo
 template <int C, int KT>
 cudaError_t launch_bwd_scalar(const float *params, const void *grad_image, const Geom &g,
                               const Workspace &ws, float *grad_params, cudaStream_t s) {
-    return g.bwd_threads == 128 ? launch_bwd_ck<C, KT, 128>(params, grad_image, g, ws, grad_params, s)
-                                : launch_bwd_ck<C, KT, 256>(params, grad_image, g, ws, grad_params, s);
+    return launch_bwd_ck<C, KT, 256>(params, grad_image, g, ws, grad_params, s);
 }
 
 template <int C>

@@ -319,9 +319,14 @@ def test_separate_bins_then_render_matches_one_call():
     (2, 40000, 1, 112, 144, 5),   # large frames: chunked count, two scan passes, 63 tiles
     (1, 20000, 2, 300, 240, 3),   # 285 tiles (more than one frame block takes), 20 chunks
     (1, 3000, 1, 2048, 2048, 5),  # the most tiles a frame may have (16384): 1-warp scatter blocks
+    (3, 1000, 2, 96, 160, 11),    # few frames: 256-Gaussian chunks, a ragged last chunk
+    (2, 4000, 1, 128, 128, 9),    # 512-Gaussian chunks... down to 256 for too few blocks
+    (5, 333, 4, 32, 64, 9),       # chunks shorter than a warp's slab
 ])
 def test_chunked_binning_paths(B, N, C, H, W, k):
-    """Frames too large for one binning block (count, two-level scan, scatter)."""
+    """Frames binned by the chunked kernels (count, scan with the frame's last
+    block scanning the tile totals, per-warp slab scatter), chunk sizes 256 to
+    1024 Gaussians."""
     rng = np.random.default_rng(N + H)
     p = _edge_params(rng, B, N, C, H, W, k, smean=0.2, ssd=0.3)
     g = rng.standard_normal((B, C, H, W)).astype(np.float32)
@@ -333,11 +338,13 @@ def test_chunked_binning_paths(B, N, C, H, W, k):
     (2, 4000, 1, 128, 128, 9),   # 64 tiles, 4000 ids
     (5, 333, 4, 32, 64, 9),      # 8 tiles, a ragged last warp of ids
     (2, 5000, 3, 48, 80, 7),     # 15 tiles, 5000 ids
-    (1, 980, 1, 192, 256, 5),    # 192 tiles x 31 warps: tables of exactly 48 KB + static arrays
+    (1, 980, 1, 192, 256, 5),    # 192 tiles, 16-warp frame blocks
 ])
 def test_frame_block_binning(B, N, C, H, W, k):
-    """Frames binned by one block each (up to 256 tiles), windows partly and
+    """Frames binned by one block each (up to 256 tiles; used when there are at
+    least as many frames as SMs, so B becomes 150 here), windows partly and
     wholly off the grid, ragged last warp of ids."""
+    B = 150
     rng = np.random.default_rng(B * 7 + N + W)
     p = _edge_params(rng, B, N, C, H, W, k)
     g = rng.standard_normal((B, C, H, W)).astype(np.float32)
