@@ -74,6 +74,7 @@ pdr_status make_geom(int B, int N, int C, int H, int W, int k, Geom *g) {
     g->out_vec2 = 0;
     g->out_vec4 = 0;
     g->img_dtype = PDR_F32;
+    g->stage_vec4 = 0;
     // Backward record capacity: room for the home Gaussians of a tile at 1.5x
     // the mean count (a tile with more is processed in several rounds), at
     // least one block's worth of list entries, at most 512.
@@ -293,6 +294,8 @@ pdr_status pdr_render_bwd_ex(const float *params, const void *grad_image, int gr
     const Workspace ws = carve(workspace, L);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     g.img_dtype = grad_dtype;
+    g.stage_vec4 = grad_dtype == PDR_F32 && (g.W & 3) == 0 &&
+                   (reinterpret_cast<uintptr_t>(grad_image) & 15) == 0;
     if (!workspace_holds_fwd_bins) {
         st = from_cuda(bin(params, g, ws, s));
         if (st != PDR_OK) return st;

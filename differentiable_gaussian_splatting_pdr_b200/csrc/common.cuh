@@ -48,6 +48,7 @@ struct Geom {
     int out_vec2;       // 1 if the output image allows 8-byte 2-pixel stores
     int out_vec4;       // 1 if the output image allows 16-byte 4-pixel stores
     int img_dtype;      // storage of image / dL/dI: PDR_F32, PDR_F16 or PDR_BF16
+    int stage_vec4;     // 1: dL/dI is fp32, rows of a multiple of 4 floats, 16-byte aligned
     int bwd_threads;    // threads per backward block
     int bwd_rcap;       // home records a backward block stages at most (>= its threads)
 };

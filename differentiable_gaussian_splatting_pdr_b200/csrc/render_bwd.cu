@@ -489,6 +489,84 @@ struct PairShape {
     __host__ __device__ static constexpr size_t smem(int rcap) { return HALO4 + HALO2 + sizeof(float4) * RV * rcap; }
 };
 
+// Stages dL/dI of the pair kernels' region [X0 - r, X0 + 15 + r] x rows
+// [Y0 - r, Y0 + 15 + r] (zero outside it and outside the grid) for fp32
+// storage with rows of a multiple of 4 floats and a 16-byte aligned image:
+// thread (row, j) loads the aligned float4 of columns X0 - 8 + 4j .. + 3 of
+// every channel (one vector load each; guarded scalar loads where it
+// crosses the grid's edge) and writes the parity elements whose first pixel
+// it holds, the second pixel of a pair that ends past its float4 coming from
+// the next lane (the float4 to its right).
+template <int C, int K, int NT>
+__device__ __forceinline__ void stage_pairs_vec4(const void *__restrict__ gimg, const Geom &g,
+                                                 int b, int X0, int Y0, float4 *halo4,
+                                                 float2 *halo2) {
+    using S = PairShape<C, K, NT>;
+    constexpr int R = S::R, NP4 = S::NP4, NP2 = S::NP2;
+    constexpr int NJ = (8 + kTile + R + 1 + 3) / 4;  // float4 columns from X0 - 8
+    static_assert(NJ == 8 && R <= 8, "one warp covers 4 rows of 8 float4 columns");
+    constexpr int NCH = 2 * NP4 + NP2;
+    const float *img = static_cast<const float *>(gimg);
+    for (int it0 = 0; it0 < S::ROWS * NJ; it0 += NT) {  // every lane runs every round (shuffle)
+        const int it = it0 + (int)threadIdx.x;
+        const int row = it / NJ, j = it - row * NJ;
+        const int y = Y0 - R + row;
+        const int x4 = X0 - 8 + 4 * j;
+        float v[NCH][4];
+        const bool rowin = row < S::ROWS && y >= 0 && y < g.H;
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+            v[c][0] = v[c][1] = v[c][2] = v[c][3] = 0.0f;
+            if (c < C && rowin) {
+                const float *src = img + (((size_t)b * C + c) * g.H + y) * g.W;
+                if (x4 >= 0 && x4 + 3 < g.W) {
+                    const float4 q = *reinterpret_cast<const float4 *>(src + x4);
+                    v[c][0] = q.x; v[c][1] = q.y; v[c][2] = q.z; v[c][3] = q.w;
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        if (x4 + e >= 0 && x4 + e < g.W) v[c][e] = src[x4 + e];
+                }
+            }
+            // zero outside [X0 - r, X0 + 15 + r]
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                if (x4 + e < X0 - R || x4 + e > X0 + kTile - 1 + R) v[c][e] = 0.0f;
+        }
+        // Element 0 of the float4 to the right: the next lane's (j + 1 of the
+        // same row, NT and NJ being multiples of 8).  For j = 7 it is never
+        // used: the last pair of either parity ends inside that float4.
+        float nx[NCH];
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) nx[c] = __shfl_down_sync(0xffffffffu, v[c][0], 1);
+        if (row >= S::ROWS) continue;
+        // Plane parity p's element m starts at column offset (8 - r) + p + 2m
+        // from X0 - 8; this float4 holds offsets 4j .. 4j + 3.
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+#pragma unroll
+            for (int f = 0; f < 4; ++f) {
+                if (((8 - R + p) & 1) != (f & 1)) continue;  // pairs start at this parity
+                const int m = (4 * j + f - (8 - R + p)) / 2;
+                if (4 * j + f - (8 - R + p) < 0 || m >= S::PAIRS) continue;
+                const int el = row * S::PITCH + m;
+#pragma unroll
+                for (int pl = 0; pl < NP4; ++pl) {
+                    const float lo0 = v[2 * pl][f], lo1 = v[2 * pl + 1][f];
+                    const float hi0 = f < 3 ? v[2 * pl][f < 3 ? f + 1 : 0] : nx[2 * pl];
+                    const float hi1 = f < 3 ? v[2 * pl + 1][f < 3 ? f + 1 : 0] : nx[2 * pl + 1];
+                    halo4[(p * NP4 + pl) * S::PLANE + el] = make_float4(lo0, hi0, lo1, hi1);
+                }
+                if constexpr (NP2) {
+                    const float lo = v[C - 1][f];
+                    const float hi = f < 3 ? v[C - 1][f < 3 ? f + 1 : 0] : nx[C - 1];
+                    halo2[p * S::PLANE + el] = make_float2(lo, hi);
+                }
+            }
+        }
+    }
+}
+
 template <int C, int K, int NT>
 __global__ void __launch_bounds__(NT, 896 / NT) k_bwd_pairs(const float *__restrict__ params,
                                                   const void *__restrict__ gimg, Geom g,
@@ -529,45 +607,49 @@ __global__ void __launch_bounds__(NT, 896 / NT) k_bwd_pairs(const float *__restr
     bool valid[kPer];
     load_pass<NT, kPer>(ids, L0, L1, raw, valid);
 
-    // Stage dL/dI over [X0 - r, X0 + 15 + r]^2 (zero outside the grid; the
-    // column after it, read only as the masked pixel of a last pair, is zero
-    // too): item (row, m) holds pixels RX0 + 2m + {0, 1, 2}; the even parity
-    // gets pair (0, 1), the odd parity pair (1, 2).  Two items per thread
-    // have their loads in flight together.
-    constexpr int SU = 2;
-    for (int i0 = 0; i0 < S::NIT; i0 += SU * NT) {
-        float v[SU][3][NCH];
+    if (g.stage_vec4) {
+        stage_pairs_vec4<C, K, NT>(gimg, g, b, X0, Y0, halo4, halo2);
+    } else {
+        // Stage dL/dI over [X0 - r, X0 + 15 + r]^2 (zero outside the grid; the
+        // column after it, read only as the masked pixel of a last pair, is zero
+        // too): item (row, m) holds pixels RX0 + 2m + {0, 1, 2}; the even parity
+        // gets pair (0, 1), the odd parity pair (1, 2).  Two items per thread
+        // have their loads in flight together.
+        constexpr int SU = 2;
+        for (int i0 = 0; i0 < S::NIT; i0 += SU * NT) {
+            float v[SU][3][NCH];
 #pragma unroll
-        for (int u = 0; u < SU; ++u) {
-            const int it = i0 + u * NT + tid;
-            const int row = it / S::PAIRS, m = it - row * S::PAIRS;
-            const int y = RY0 + row;
-            const bool rowin = it < S::NIT && y >= 0 && y < g.H;
+            for (int u = 0; u < SU; ++u) {
+                const int it = i0 + u * NT + tid;
+                const int row = it / S::PAIRS, m = it - row * S::PAIRS;
+                const int y = RY0 + row;
+                const bool rowin = it < S::NIT && y >= 0 && y < g.H;
 #pragma unroll
-            for (int q = 0; q < 3; ++q) {
-                const int x = RX0 + 2 * m + q;
-                const bool in = rowin && x >= 0 && x < g.W && x <= X0 + kTile - 1 + R;
+                for (int q = 0; q < 3; ++q) {
+                    const int x = RX0 + 2 * m + q;
+                    const bool in = rowin && x >= 0 && x < g.W && x <= X0 + kTile - 1 + R;
 #pragma unroll
-                for (int c = 0; c < NCH; ++c)
-                    v[u][q][c] = (in && c < C) ? img_load(gimg, (((size_t)b * C + c) * g.H + y) * g.W + x, g.img_dtype) : 0.0f;
+                    for (int c = 0; c < NCH; ++c)
+                        v[u][q][c] = (in && c < C) ? img_load(gimg, (((size_t)b * C + c) * g.H + y) * g.W + x, g.img_dtype) : 0.0f;
+                }
             }
-        }
 #pragma unroll
-        for (int u = 0; u < SU; ++u) {
-            const int it = i0 + u * NT + tid;
-            if (it >= S::NIT) continue;
-            const int row = it / S::PAIRS, m = it - row * S::PAIRS;
-            const int el = row * S::PITCH + m;
+            for (int u = 0; u < SU; ++u) {
+                const int it = i0 + u * NT + tid;
+                if (it >= S::NIT) continue;
+                const int row = it / S::PAIRS, m = it - row * S::PAIRS;
+                const int el = row * S::PITCH + m;
 #pragma unroll
-            for (int pl = 0; pl < NP4; ++pl) {
-                halo4[pl * S::PLANE + el] = make_float4(v[u][0][2 * pl], v[u][1][2 * pl],
-                                                        v[u][0][2 * pl + 1], v[u][1][2 * pl + 1]);
-                halo4[(NP4 + pl) * S::PLANE + el] = make_float4(v[u][1][2 * pl], v[u][2][2 * pl],
-                                                                v[u][1][2 * pl + 1], v[u][2][2 * pl + 1]);
-            }
-            if constexpr (NP2) {
-                halo2[el] = make_float2(v[u][0][C - 1], v[u][1][C - 1]);
-                halo2[S::PLANE + el] = make_float2(v[u][1][C - 1], v[u][2][C - 1]);
+                for (int pl = 0; pl < NP4; ++pl) {
+                    halo4[pl * S::PLANE + el] = make_float4(v[u][0][2 * pl], v[u][1][2 * pl],
+                                                            v[u][0][2 * pl + 1], v[u][1][2 * pl + 1]);
+                    halo4[(NP4 + pl) * S::PLANE + el] = make_float4(v[u][1][2 * pl], v[u][2][2 * pl],
+                                                                    v[u][1][2 * pl + 1], v[u][2][2 * pl + 1]);
+                }
+                if constexpr (NP2) {
+                    halo2[el] = make_float2(v[u][0][C - 1], v[u][1][C - 1]);
+                    halo2[S::PLANE + el] = make_float2(v[u][1][C - 1], v[u][2][C - 1]);
+                }
             }
         }
     }

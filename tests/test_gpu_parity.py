@@ -370,15 +370,18 @@ def test_knob_workloads(name):
 
 
 @pytest.mark.parametrize("dtype,bar", [("float16", 1e-3), ("bfloat16", 8e-3)])
-@pytest.mark.parametrize("name", ["mono64", "rgb128", "field32x64"])
+@pytest.mark.parametrize("name", ["mono64", "rgb128", "field32x64", "stress512-small"])
 def test_reduced_precision_storage(name, dtype, bar):
     """Image and dL/dI stored as fp16 / bf16, sums in fp32: the stored image is
     the fp32 image rounded once; gradients from a half-precision dL/dI match the
-    oracle given the same (widened) values at the fp32 bar."""
+    oracle given the same (widened) values at the fp32 bar.  stress512-small
+    (one 96 x 128 frame of stress512's distributions, k = 15) takes the
+    pixel-pair backward with its element-wise dL/dI staging."""
     import torch
     from differentiable_gaussian_splatting_pdr_b200 import api as R
     tdt = getattr(torch, dtype)
-    w = WORKLOADS[name]
+    w = (WORKLOADS["stress512"].scaled(B=1, H=96, W=128, N=3072) if name == "stress512-small"
+         else WORKLOADS[name])
     p, g = make_inputs(w)
     dev = torch.device("cuda:0")
     pt = torch.from_numpy(p).to(dev)
