@@ -12,15 +12,13 @@ namespace pdr {
 namespace {
 
 constexpr size_t kAlign = 256;
-constexpr size_t kScatterSmemLimit = 200 * 1024;
-constexpr int kScatterWarps = 8;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 
 int tiles_per_axis(int k) { return (k - 1 + kTile - 1) / kTile + 1; }
 
 struct Layout {
-    size_t err, gr, hist, offs, ids, total;
+    size_t err, gr, hist, tot, offs, ids, total;
 };
 
 pdr_status make_geom(int B, int N, int C, int H, int W, int k, Geom *g) {
@@ -41,22 +39,32 @@ pdr_status make_geom(int B, int N, int C, int H, int W, int k, Geom *g) {
     g->P = 5 + C;
     g->m = (int)m;
     g->cap = (int)cap;
-    // Chunks of 1024 Gaussians, halved (down to 256) while the launch would
-    // have fewer than two binning blocks per SM.
+    // Binning slabs of 32 * R Gaussians (one scatter warp each): R = 8, halved
+    // while the frames would give fewer than eight scatter warps per SM, but
+    // at least T / 128 so that the per-slab counts (B x slabs x T ints) stay
+    // within about four ints per Gaussian.  Slabs under 256 Gaussians divide
+    // 256 (R = 1, 2, 4).
     {
-        int ch = kBinChunk;
-        while (ch > kBinChunkMin && (long long)B * ((N + ch - 1) / ch) < 2 * 148) ch >>= 1;
-        g->chunk = ch;
-        g->nchunks = (N + ch - 1) / ch;
+        int R = 8;
+        while (R > 1 && (long long)B * ((N + 32 * R - 1) / (32 * R)) < 8 * 148) R >>= 1;
+        int rmin = (int)((T + 127) / 128);
+        if (rmin <= 8) rmin = rmin <= 1 ? 1 : rmin <= 2 ? 2 : rmin <= 4 ? 4 : 8;  // divides 256
+        if (R < rmin) R = rmin;
+        g->slab = 32 * R;
+        g->nslab = (N + g->slab - 1) / g->slab;
     }
-    int nw = kScatterWarps;  // scatter block: as many warps as the per-warp tile tables allow
-    while (nw > 1 && (size_t)T * (6 * nw + 4) + 16 > kScatterSmemLimit) nw >>= 1;
-    if ((size_t)T * (6 * nw + 4) + 16 > kScatterSmemLimit) return PDR_ERR_TOO_LARGE;
-    g->scatter_warps = nw;
+    if (m > 3) return PDR_ERR_TOO_LARGE;  // the slab scatter handles windows over at most 3 tiles per axis
+    // Slab-scatter block: up to 8 warps while its tables (a list start per
+    // tile, and a slot and a mask table per warp) stay within 100 KB.
+    {
+        int nw = 8;
+        while (nw > 1 && (size_t)T * 4 * (1 + 2 * nw) > 100 * 1024) nw >>= 1;
+        g->slab_warps = nw;  // one warp: 12 bytes per tile, <= 192 KB for the most tiles
+    }
     // Small frames: one binning block per frame (its shared-memory tables
     // hold [2 + 2 * warps] x T ints).
     // (only when the frames alone give at least one block per SM; otherwise
-    // the chunked kernels spread the work over more blocks)
+    // the slab kernels spread the work over more blocks)
     g->frame_block = T <= kFrameBlockMaxT && N <= kFrameBlockMaxN && B >= 148;
     int ft = ((N + 31) / 32) * 32;
     if (ft > 1024) ft = 1024;
@@ -95,9 +103,10 @@ pdr_status make_geom(int B, int N, int C, int H, int W, int k, Geom *g) {
 Layout make_layout(const Geom &g) {
     Layout L;
     size_t o = 0;
-    L.err = o; o += align_up(sizeof(int) * (1 + (size_t)g.B));  // error word, then the scan counters
+    L.err = o; o += align_up(sizeof(int));  // the device error word
     L.gr = o; o += align_up(sizeof(float4) * 2 * (size_t)g.B * g.N);
-    L.hist = o; o += align_up(sizeof(int) * (size_t)g.B * g.nchunks * g.T);
+    L.hist = o; o += align_up(sizeof(int) * (size_t)g.B * g.nslab * g.T);
+    L.tot = o; o += align_up(sizeof(int) * (size_t)g.B * g.T);
     L.offs = o; o += align_up(sizeof(int) * (size_t)g.B * (g.T + 1));
     L.ids = o; o += align_up(sizeof(int) * (size_t)g.B * g.cap);
     L.total = o;
@@ -108,9 +117,9 @@ Workspace carve(void *base, const Layout &L) {
     char *p = static_cast<char *>(base);
     Workspace w;
     w.err = reinterpret_cast<int *>(p + L.err);
-    w.done = w.err + 1;
     w.gr = reinterpret_cast<float4 *>(p + L.gr);
     w.hist = reinterpret_cast<int *>(p + L.hist);
+    w.tot = reinterpret_cast<int *>(p + L.tot);
     w.offs = reinterpret_cast<int *>(p + L.offs);
     w.ids = reinterpret_cast<int *>(p + L.ids);
     return w;
@@ -164,13 +173,8 @@ cudaError_t clear_error_word(const Workspace &ws, cudaStream_t s) {
     return cudaMemsetAsync(ws.err, 0, sizeof(int), s);
 }
 
-// The error word and the tile scan's per-frame counters, cleared together.
-cudaError_t clear_error_and_counters(const Geom &g, const Workspace &ws, cudaStream_t s) {
-    return cudaMemsetAsync(ws.err, 0, sizeof(int) * (1 + (size_t)g.B), s);
-}
-
 cudaError_t bin(const float *params, const Geom &g, const Workspace &ws, cudaStream_t s) {
-    cudaError_t e = clear_error_and_counters(g, ws, s);
+    cudaError_t e = clear_error_word(ws, s);
     if (e != cudaSuccess) return e;
     if (g.N == 0)  // no Gaussians: every tile list empty at 0
         return cudaMemsetAsync(ws.offs, 0, sizeof(int) * (size_t)g.B * (g.T + 1), s);

@@ -2,23 +2,19 @@
 // clipped k x k window touches, lists in ascending Gaussian id so that every
 // fp32 sum downstream has a fixed order.  The additive accumulation (reading
 // notes, "Method") has no depth order, so any fixed order is correct;
-// ascending id is the one the oracle also uses.  Three kernels on the
-// caller's stream, no float atomics, no host synchronisation:
+// ascending id is the one the oracle also uses.  No float atomics, no host
+// synchronisation; integer shared-memory atomics only count or set lane bits,
+// never decide a position.
 //
-//   k_count   one block per (frame, chunk of 256 .. 1024 Gaussians): the
-//             per-Gaussian record (window centre, rotated and scaled axes)
-//             and the chunk's per-tile counts (integer shared-memory atomics
-//             count only; they never decide a position);
-//   k_scan_tiles
-//             exclusive prefix of each tile's counts over the chunks (32 tiles
-//             x 32 chunks per step through shared memory); the last block of
-//             a frame to finish scans the frame's tile totals into the tiles'
-//             list starts;
-//   k_scatter one block per (frame, chunk): stable ranks in rounds of
-//             blockDim Gaussians -- rank in a tile = earlier chunks (the scans) +
-//             earlier rounds + earlier warps' popcounts + lanes below in this
-//             warp (per-warp lane bitmasks) -- so positions never depend on
-//             the order in which atomics land.
+// Large frames (three kernels on the caller's stream; a slab is g.slab
+// consecutive Gaussians of a frame, one warp each):
+//   k_slab_count    per slab: the per-Gaussian records (window centre,
+//                   rotated and scaled axes) and the slab's count per tile;
+//   k_slab_scan     per tile: exclusive prefix of the counts over the slabs,
+//                   and the tile's total;
+//   k_slab_scatter  per block: the tiles' list starts (block scan of the
+//                   totals); per slab: stable ranks in rounds of 32 from
+//                   lane masks, written at start + slab prefix + rank.
 // Small frames (g.frame_block) take one launch instead: k_bin_frame, one
 // block per frame, does the records, the counts, the tile offsets and the
 // stable scatter in shared memory (ranks from a per-tile prefix over the
@@ -29,151 +25,18 @@ namespace pdr {
 
 namespace {
 
-constexpr int kCountThreads = 256;
-
-__global__ void __launch_bounds__(kCountThreads) k_count(const float *__restrict__ params,
-                                                         Geom g, float4 *__restrict__ gr,
-                                                         int *__restrict__ hist,
-                                                         int *__restrict__ err) {
-    extern __shared__ int hs[];  // [T]
-    const int b = blockIdx.y, c = blockIdx.x;
-    for (int t = threadIdx.x; t < g.T; t += blockDim.x) hs[t] = 0;
-    __syncthreads();
-    const int i0 = c * g.chunk, i1 = min(i0 + g.chunk, g.N);
-    constexpr int U = kBinChunk / kCountThreads;  // Gaussians per thread at most, all in flight
-    float4 A[U], Q[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-        const int i = i0 + u * kCountThreads + threadIdx.x;
-        if (i < i1) gaussian_record(params + ((size_t)b * g.N + i) * g.P, A[u], Q[u]);
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-        const int i = i0 + u * kCountThreads + threadIdx.x;
-        if (i >= i1) continue;
-        const size_t gid = (size_t)b * g.N + i;
-        gr[2 * gid] = A[u];
-        gr[2 * gid + 1] = Q[u];
-        int x0, x1, y0, y1;
-        if (window_rect(__float_as_int(Q[u].z), __float_as_int(Q[u].w), g, x0, x1, y0, y1)) {
-            for (int ty = y0 >> 4; ty <= (y1 >> 4); ++ty)
-                for (int tx = x0 >> 4; tx <= (x1 >> 4); ++tx) atomicAdd(&hs[ty * g.TX + tx], 1);
-        }
-    }
-    __syncthreads();
-    int *h = hist + ((size_t)b * g.nchunks + c) * g.T;
-    for (int t = threadIdx.x; t < g.T; t += blockDim.x) h[t] = hs[t];
-}
-
-// Block-wide inclusive scan of one int per thread (blockDim.x a multiple of 32).
-__device__ __forceinline__ int block_incl_scan(int v, int *warp_tot, int &total) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int nw = blockDim.x >> 5;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-        const int u = __shfl_up_sync(0xffffffffu, v, d);
-        if (lane >= d) v += u;
-    }
-    if (lane == 31) warp_tot[warp] = v;
-    __syncthreads();
-    if (warp == 0) {
-        int w = lane < nw ? warp_tot[lane] : 0;
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            const int u = __shfl_up_sync(0xffffffffu, w, d);
-            if (lane >= d) w += u;
-        }
-        if (lane < nw) warp_tot[lane] = w;
-    }
-    __syncthreads();
-    total = warp_tot[nw - 1];
-    const int r = v + (warp ? warp_tot[warp - 1] : 0);
-    __syncthreads();
-    return r;
-}
-
-// hist[b][c][t] <- exclusive prefix over c of the counts (relative to the
-// tile's list start); offs[b][t] <- the tile's list start.  Block (x, b)
-// takes tiles 32x .. 32x + 31 of frame b: the chunk counts pass through
-// shared memory 32 chunks at a time (coalesced along the tiles on both
-// sides), and warp w scans tile 32x + w over those chunks, carrying the
-// running sum; the tile totals go to offs[b][t].  The last block of frame b
-// to finish (a counter in the workspace, zeroed before the binner runs;
-// nothing waits on it) then scans the frame's tile totals into list starts.
-__global__ void __launch_bounds__(1024) k_scan_tiles(Geom g, int *__restrict__ hist,
-                                                     int *__restrict__ offs,
-                                                     int *__restrict__ done) {
-    __shared__ int v[32][33];  // [chunk][tile], padded against bank conflicts
-    __shared__ int warp_tot[32];
-    __shared__ int last;
-    const int b = blockIdx.y, t0 = blockIdx.x * 32;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int *h = hist + (size_t)b * g.nchunks * g.T;
-    int carry = 0;  // warp's tile: sum of the chunks already scanned
-    for (int c0 = 0; c0 < g.nchunks; c0 += 32) {
-        {
-            const int c = c0 + warp, t = t0 + lane;  // load: warp = chunk, lane = tile
-            v[warp][lane] = (c < g.nchunks && t < g.T) ? h[(size_t)c * g.T + t] : 0;
-        }
-        __syncthreads();
-        {
-            const int x = v[lane][warp];  // scan: warp = tile, lane = chunk
-            int incl = x;
-#pragma unroll
-            for (int d = 1; d < 32; d <<= 1) {
-                const int u = __shfl_up_sync(0xffffffffu, incl, d);
-                if (lane >= d) incl += u;
-            }
-            v[lane][warp] = carry + incl - x;
-            carry += __shfl_sync(0xffffffffu, incl, 31);
-        }
-        __syncthreads();
-        {
-            const int c = c0 + warp, t = t0 + lane;
-            if (c < g.nchunks && t < g.T) h[(size_t)c * g.T + t] = v[warp][lane];
-        }
-        __syncthreads();
-    }
-    int *o = offs + (size_t)b * (g.T + 1);
-    if (lane == 0 && t0 + warp < g.T) {
-        o[t0 + warp] = carry;
-        __threadfence();  // this total is visible before the block is counted
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) last = atomicAdd(&done[b], 1) == (int)gridDim.x - 1;
-    __syncthreads();
-    if (!last) return;
-    __threadfence();
-    int fcarry = b * g.cap;
-    for (int s0 = 0; s0 < g.T; s0 += blockDim.x) {
-        const int t = s0 + threadIdx.x;
-        const int tot = t < g.T ? __ldcg(o + t) : 0;
-        int total;
-        const int incl = block_incl_scan(tot, warp_tot, total);
-        if (t < g.T) o[t] = fcarry + incl - tot;
-        fcarry += total;
-    }
-    if (threadIdx.x == 0) {
-        o[g.T] = fcarry;
-        done[b] = 0;
-    }
-}
-
-// Stable scatter of one chunk: warp w of the block owns the contiguous slab
-// [c * chunk + w * S, + S) of the chunk (S = chunk / warps), so list
-// order = (warp, sub-round of 32, lane) = ascending id.  Each lane loads the
-// window centres of all its Gaussians first (every load in flight at once)
-// and keeps them in registers for both passes:
-//   pass 1: per-(warp, tile) entry counts (shared-memory atomics that only
-//           count, never decide a position);
-//   prefix: each warp's first slot per tile, relative to the chunk's start
-//           in that tile's list, from the counts of the earlier warps;
+// Stable scatter of a frame by the block's warps (k_bin_frame): warp w owns
+// the contiguous slab [w * S, (w + 1) * S) of the frame, so list order =
+// (warp, sub-round of 32, lane) = ascending id.
+//   pass 1: per-(warp, tile) entry counts;
+//   prefix: each warp's first slot per tile, relative to the tile's start,
+//           from the counts of the earlier warps;
 //   pass 2: each warp walks its slab again, 32 Gaussians at a time: the lane
 //           bits of a warp-private mask per tile give the rank among this
 //           sub-round's lanes, the warp's running slot per tile gives the
 //           rest.  Only warp-level synchronisation inside the passes.
 // The entry of each Gaussian in the list of its home tile carries kHomeFlag.
-constexpr int kScatterSub = 8;  // sub-rounds of 32 per warp at most (S <= 256)
+constexpr int kScatterSub = 8;  // sub-rounds of 32 whose centres a lane holds
 
 __device__ __forceinline__ void scatter_sub(const Geom &g, int b, int i, int cx, int cy,
                                             unsigned *mym, unsigned short *myslot,
@@ -280,35 +143,223 @@ __device__ __forceinline__ void warp_prefix(int T, int nw, unsigned *masks, unsi
     }
 }
 
-__global__ void k_scatter(Geom g, const float4 *__restrict__ gr, const int *__restrict__ hist,
-                          const int *__restrict__ offs, int *__restrict__ ids,
-                          int *__restrict__ err) {
-    extern __shared__ unsigned sm[];
-    const int nw = blockDim.x >> 5, T = g.T;
-    unsigned *masks = sm;                                                        // [nw][T]
-    int *tbase = reinterpret_cast<int *>(sm + nw * T);                          // [T]
-    unsigned short *slots = reinterpret_cast<unsigned short *>(tbase + T);      // [nw][T]
-    const int b = blockIdx.y, c = blockIdx.x;
-    const int warp = threadIdx.x >> 5;
-    for (int t = threadIdx.x; t < nw * T; t += blockDim.x) masks[t] = 0u;  // pass-1 counters
-    const int *hsrc = hist + ((size_t)b * g.nchunks + c) * T;
-    const int *osrc = offs + (size_t)b * (T + 1);
-    for (int t = threadIdx.x; t < T; t += blockDim.x) tbase[t] = osrc[t] + hsrc[t];
-    const int S = g.chunk / nw;
-    const int c0 = c * g.chunk, c1 = min(c0 + g.chunk, g.N);
-    const int i0 = min(c0 + warp * S, c1), i1 = min(i0 + S, c1);
-    const bool resident = S <= 32 * kScatterSub;
-    int cx[kScatterSub], cy[kScatterSub];
-    if (resident) load_centres(g, gr, b, i0, i1, cx, cy);
+// ---- large frames: the slab binner ---------------------------------------
+// A slab is g.slab consecutive Gaussians of one frame (a multiple of 32):
+// counted by k_slab_count blocks of 256 threads, scattered by one warp of
+// k_slab_scatter in rounds of 32.
+constexpr int kSlabThreads = 256;
+constexpr int kSlabWarps = 8;  // most warps (slabs) per k_slab_scatter block
+
+// Window of a Gaussian as a tile rectangle: tiles (tx0 + dx, ty0 + dy) for
+// dx < nx, dy < ny (nx = ny = 0 when the window misses the grid).
+__device__ __forceinline__ void window_tiles(int cx, int cy, const Geom &g, int &tx0, int &ty0,
+                                             int &nx, int &ny) {
+    int x0, x1, y0, y1;
+    if (window_rect(cx, cy, g, x0, x1, y0, y1)) {
+        tx0 = x0 >> 4;
+        ty0 = y0 >> 4;
+        nx = (x1 >> 4) - tx0 + 1;
+        ny = (y1 >> 4) - ty0 + 1;
+    } else {
+        tx0 = ty0 = nx = ny = 0;
+    }
+}
+
+// Per slab: the records of its Gaussians (written to gr) and its entry
+// count per tile, hist[b][s][t].  A block takes max(slab, 256) consecutive
+// Gaussians, one per thread and round: one slab, or 256 / slab whole slabs
+// (one shared-memory count table each).  Grid (ceil(N / max(slab, 256)), B).
+__global__ void __launch_bounds__(kSlabThreads) k_slab_count(const float *__restrict__ params,
+                                                             Geom g, float4 *__restrict__ gr,
+                                                             int *__restrict__ hist) {
+    extern __shared__ int cnt[];  // [slabs of the block][T]
+    const int T = g.T, b = blockIdx.y;
+    const int span = max(g.slab, kSlabThreads), ntab = span / g.slab;
+    const int s0 = blockIdx.x * ntab;  // first slab of the block
+    for (int t = threadIdx.x; t < ntab * T; t += kSlabThreads) cnt[t] = 0;
     __syncthreads();
-    int *mycnt = reinterpret_cast<int *>(masks + warp * T);
-    unsigned *mym = masks + warp * T;
-    unsigned short *myslot = slots + warp * T;
-    slab_pass(g, gr, b, i0, i1, 1, cx, cy, resident, mycnt, mym, myslot, tbase, ids, err);
+    int *mine = cnt + (ntab > 1 ? (int)threadIdx.x / g.slab : 0) * T;
+    const int i1 = min((blockIdx.x + 1) * span, g.N);
+    for (int i = blockIdx.x * span + threadIdx.x; i < i1; i += kSlabThreads) {
+        const size_t gid = (size_t)b * g.N + i;
+        float4 A, Q;
+        gaussian_record(params + gid * g.P, A, Q);
+        gr[2 * gid] = A;
+        gr[2 * gid + 1] = Q;
+        int tx0, ty0, nx, ny;
+        window_tiles(__float_as_int(Q.z), __float_as_int(Q.w), g, tx0, ty0, nx, ny);
+        for (int dy = 0; dy < ny; ++dy)
+            for (int dx = 0; dx < nx; ++dx) atomicAdd(&mine[(ty0 + dy) * g.TX + tx0 + dx], 1);
+    }
     __syncthreads();
-    warp_prefix(T, nw, masks, slots);
+    for (int q = threadIdx.x; q < ntab * T; q += kSlabThreads) {
+        const int tab = q / T, s = s0 + tab;
+        if (s < g.nslab) hist[((size_t)b * g.nslab + s) * T + (q - tab * T)] = cnt[q];
+    }
+}
+
+// hist[b][s][t] <- exclusive prefix over the slabs s (the slab's first slot
+// in tile t, relative to the tile's list start); tot[b][t] <- the tile's
+// entry count.  Block (x, b) takes tiles 32x .. 32x + 31 of frame b, lane =
+// tile (coalesced rows); warp w takes a contiguous run of slabs, sums it,
+// the 32 x 32 partial sums are scanned across the warps through shared
+// memory, and each warp rescans its run from its offset.  Runs of at most
+// kScanRegs slabs stay in registers between the two sweeps.
+constexpr int kScanRegs = 8;
+
+__global__ void __launch_bounds__(1024) k_slab_scan(Geom g, int *__restrict__ hist,
+                                                    int *__restrict__ tot) {
+    __shared__ int part[32][33];  // [warp][tile], padded against bank conflicts
+    const int b = blockIdx.y, t0 = blockIdx.x * 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int t = t0 + lane, T = g.T;
+    const bool tin = t < T;
+    const int spw = (g.nslab + 31) / 32;
+    const int s0 = min(warp * spw, g.nslab), s1 = min(s0 + spw, g.nslab);
+    int *h = hist + (size_t)b * g.nslab * T + t;
+    const bool inreg = spw <= kScanRegs;  // block-uniform
+    int x[kScanRegs];
+    int sum = 0;
+    if (inreg) {
+#pragma unroll
+        for (int q = 0; q < kScanRegs; ++q) {
+            x[q] = (s0 + q < s1 && tin) ? h[(size_t)(s0 + q) * T] : 0;
+            sum += x[q];
+        }
+    } else if (tin) {
+        for (int s = s0; s < s1; ++s) sum += h[(size_t)s * T];
+    }
+    part[warp][lane] = sum;
     __syncthreads();
-    slab_pass(g, gr, b, i0, i1, 2, cx, cy, resident, mycnt, mym, myslot, tbase, ids, err);
+    {
+        // warp = tile, lane = slab run
+        const int v = part[lane][warp];
+        int incl = v;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int u = __shfl_up_sync(0xffffffffu, incl, d);
+            if (lane >= d) incl += u;
+        }
+        part[lane][warp] = incl - v;
+        if (lane == 31 && t0 + warp < T) tot[(size_t)b * T + t0 + warp] = incl;
+    }
+    __syncthreads();
+    if (!tin) return;
+    int run = part[warp][lane];
+    if (inreg) {
+#pragma unroll
+        for (int q = 0; q < kScanRegs; ++q)
+            if (s0 + q < s1) {
+                h[(size_t)(s0 + q) * T] = run;
+                run += x[q];
+            }
+    } else {
+        for (int s = s0; s < s1; ++s) {
+            const int v = h[(size_t)s * T];
+            h[(size_t)s * T] = run;
+            run += v;
+        }
+    }
+}
+
+// Stable scatter, one warp per slab, grid (ceil(nslab / slab_warps), B).  The
+// block first turns the frame's tile totals into list starts (a block scan;
+// block 0 of the frame also publishes them in offs).  Warp w then keeps two
+// tables over the tiles: the next free slot of its slab in each tile (list
+// start + the slab's exclusive prefix) and a lane mask.  Per round of 32
+// Gaussians (lane = id order): every lane sets its bit in the masks of its
+// tiles; its rank in a tile is the number of lower lanes in that mask; the
+// lowest lane of each tile then advances the tile's slot by the mask's
+// population and clears the mask.  List order = (slab, round, lane) =
+// ascending id, whatever order the shared-memory atomics land in.  The
+// entry in the list of the Gaussian's home tile carries kHomeFlag.
+template <int M>  // most tiles a window touches along an axis (2: k <= 17, 3: k <= 33)
+__global__ void __launch_bounds__(32 * kSlabWarps) k_slab_scatter(
+    Geom g, const float4 *__restrict__ gr, const int *__restrict__ hist,
+    const int *__restrict__ tot, int *__restrict__ offs, int *__restrict__ ids,
+    int *__restrict__ err) {
+    extern __shared__ int ssm[];
+    __shared__ int warp_tot[32];
+    const int T = g.T, nwb = blockDim.x >> 5;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int b = blockIdx.y, s = blockIdx.x * nwb + warp;
+    int *fofs = ssm;  // [T] list starts of the frame's tiles
+    {
+        // Thread j sums tiles [j * Q, j * Q + Q); one block scan.
+        const int Q = (T + (int)blockDim.x - 1) / (int)blockDim.x;
+        const int *tb = tot + (size_t)b * T;
+        const int ta = min((int)threadIdx.x * Q, T), tz = min(ta + Q, T);
+        int sum = 0;
+        for (int t = ta; t < tz; ++t) sum += tb[t];
+        int total;
+        int run = b * g.cap + block_excl_scan(sum, warp_tot, total);
+        for (int t = ta; t < tz; ++t) {
+            fofs[t] = run;
+            run += tb[t];
+        }
+        if (blockIdx.x == 0 && threadIdx.x == 0) offs[(size_t)b * (T + 1) + T] = b * g.cap + total;
+    }
+    __syncthreads();
+    if (blockIdx.x == 0) {
+        int *o = offs + (size_t)b * (T + 1);
+        for (int t = threadIdx.x; t < T; t += blockDim.x) o[t] = fofs[t];
+    }
+    if (s >= g.nslab) return;  // warp-uniform, after the last block barrier
+    int *nxt = ssm + T + warp * 2 * T;
+    unsigned *msk = reinterpret_cast<unsigned *>(nxt + T);
+    const int *h = hist + ((size_t)b * g.nslab + s) * T;
+    for (int t = lane; t < T; t += 32) {
+        nxt[t] = fofs[t] + h[t];
+        msk[t] = 0u;
+    }
+    __syncwarp();
+    const unsigned lt = lanemask_lt();
+    const int lo = b * g.cap, hi = lo + g.cap;
+    const int i0 = s * g.slab, i1 = min(i0 + g.slab, g.N);
+    for (int g0 = i0; g0 < i1; g0 += 32 * kScatterSub) {
+        int cx[kScatterSub], cy[kScatterSub];
+        load_centres(g, gr, b, g0, i1, cx, cy);
+#pragma unroll
+        for (int j = 0; j < kScatterSub; ++j) {
+            if (g0 + 32 * j >= i1) break;  // warp-uniform
+            const int i = g0 + 32 * j + lane;  // past i1: no centre, no tiles
+            int tx0, ty0, nx, ny;
+            window_tiles(cx[j], cy[j], g, tx0, ty0, nx, ny);
+            const int ht = nx ? home_tile(cx[j], cy[j], g) : -1;
+            int tk[M * M];
+#pragma unroll
+            for (int dy = 0; dy < M; ++dy)
+#pragma unroll
+                for (int dx = 0; dx < M; ++dx) {
+                    const int q = dy * M + dx;
+                    tk[q] = (dx < nx && dy < ny) ? (ty0 + dy) * g.TX + tx0 + dx : -1;
+                    if (tk[q] >= 0) atomicOr(&msk[tk[q]], 1u << lane);
+                }
+            __syncwarp();
+            int nb[M * M];
+#pragma unroll
+            for (int q = 0; q < M * M; ++q) {
+                nb[q] = -1;
+                if (tk[q] < 0) continue;
+                const unsigned m = msk[tk[q]];
+                const int base = nxt[tk[q]];
+                const int slot = base + __popc(m & lt);
+                if (slot >= lo && slot < hi)
+                    ids[slot] = (int)((unsigned)i | (tk[q] == ht ? kHomeFlag : 0u));
+                else
+                    atomicOr(err, kErrListBounds);
+                if ((m & lt) == 0u) nb[q] = base + __popc(m);  // lowest lane of the tile
+            }
+            __syncwarp();
+#pragma unroll
+            for (int q = 0; q < M * M; ++q)
+                if (nb[q] >= 0) {
+                    nxt[tk[q]] = nb[q];
+                    msk[tk[q]] = 0u;
+                }
+            __syncwarp();
+        }
+    }
 }
 
 // One block per frame: the whole binner of a small frame in one launch.
@@ -409,40 +460,52 @@ static size_t bin_tables_bytes(int T, int nw) { return (size_t)T * (6 * (size_t)
 
 size_t bin_frame_smem(const Geom &g) { return bin_tables_bytes(g.T, g.frame_threads / 32); }
 
-size_t bin_count_smem(const Geom &g) { return sizeof(int) * (size_t)g.T; }
+// k_slab_count: one count per tile; k_slab_scatter: the tiles' list starts,
+// then a slot and a mask table per warp.
+size_t bin_count_smem(const Geom &g) {
+    const int ntab = g.slab < kSlabThreads ? kSlabThreads / g.slab : 1;
+    return sizeof(int) * (size_t)g.T * ntab;
+}
 
-size_t bin_scatter_smem(const Geom &g) { return bin_tables_bytes(g.T, g.scatter_warps); }
+size_t bin_scatter_smem(const Geom &g) {
+    return sizeof(int) * (size_t)g.T * (1 + 2 * (size_t)g.slab_warps);
+}
 
 // Dynamic shared memory above which a launch needs the opt-in attribute: the
 // 48 KB default less room for the kernel's static arrays.
 constexpr size_t kStaticSmemRoom = 44 * 1024;
+
+template <typename K>
+static cudaError_t allow_smem(K kernel, size_t bytes) {
+    if (bytes <= kStaticSmemRoom) return cudaSuccess;
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
 
 cudaError_t launch_bin(const float *params, const Geom &g, const Workspace &ws,
                        cudaStream_t s) {
     cudaError_t e;
     if (g.frame_block) {
         const size_t sf = bin_frame_smem(g);
-        if (sf > kStaticSmemRoom) {
-            e = cudaFuncSetAttribute(k_bin_frame, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)sf);
-            if (e != cudaSuccess) return e;
-        }
+        if ((e = allow_smem(k_bin_frame, sf)) != cudaSuccess) return e;
         k_bin_frame<<<g.B, g.frame_threads, sf, s>>>(params, g, ws.gr, ws.offs, ws.ids, ws.err);
         return cudaGetLastError();
     }
     const size_t sc = bin_count_smem(g), ss = bin_scatter_smem(g);
-    if (sc > 48 * 1024) {
-        e = cudaFuncSetAttribute(k_count, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sc);
-        if (e != cudaSuccess) return e;
+    if ((e = allow_smem(k_slab_count, sc)) != cudaSuccess) return e;
+    const int span = g.slab > kSlabThreads ? g.slab : kSlabThreads;
+    k_slab_count<<<dim3((g.N + span - 1) / span, g.B), kSlabThreads, sc, s>>>(params, g, ws.gr,
+                                                                            ws.hist);
+    k_slab_scan<<<dim3((g.T + 31) / 32, g.B), 1024, 0, s>>>(g, ws.hist, ws.tot);
+    const dim3 grid((g.nslab + g.slab_warps - 1) / g.slab_warps, g.B);
+    if (g.m <= 2) {
+        if ((e = allow_smem(k_slab_scatter<2>, ss)) != cudaSuccess) return e;
+        k_slab_scatter<2><<<grid, 32 * g.slab_warps, ss, s>>>(g, ws.gr, ws.hist, ws.tot, ws.offs,
+                                                               ws.ids, ws.err);
+    } else {
+        if ((e = allow_smem(k_slab_scatter<3>, ss)) != cudaSuccess) return e;
+        k_slab_scatter<3><<<grid, 32 * g.slab_warps, ss, s>>>(g, ws.gr, ws.hist, ws.tot, ws.offs,
+                                                               ws.ids, ws.err);
     }
-    if (ss > 48 * 1024) {
-        e = cudaFuncSetAttribute(k_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ss);
-        if (e != cudaSuccess) return e;
-    }
-    const dim3 grid(g.nchunks, g.B);
-    k_count<<<grid, kCountThreads, sc, s>>>(params, g, ws.gr, ws.hist, ws.err);
-    k_scan_tiles<<<dim3((g.T + 31) / 32, g.B), 1024, 0, s>>>(g, ws.hist, ws.offs, ws.done);
-    k_scatter<<<grid, 32 * g.scatter_warps, ss, s>>>(g, ws.gr, ws.hist, ws.offs, ws.ids, ws.err);
     return cudaGetLastError();
 }
 

@@ -38,9 +38,9 @@ struct Geom {
     int P;              // parameters per Gaussian (5 + C)
     int m;              // most tiles a window can touch along one axis
     int cap;            // tile-list capacity per frame (N * m * m)
-    int chunk;          // Gaussians per binning chunk (a power of two, <= kBinChunk)
-    int nchunks;        // binning chunks per frame
-    int scatter_warps;  // warps per scatter block
+    int slab;           // Gaussians per binning slab (32, 64, 128 or a multiple of 256)
+    int nslab;          // binning slabs per frame
+    int slab_warps;     // warps (slabs) per block of the slab scatter
     int frame_block;    // 1: small frames, one binning block per frame
     int frame_threads;  // threads of that block
     int cluster_fwd;    // 1: frames of <= kClusterTiles tiles, bins + forward in one launch
@@ -53,8 +53,6 @@ struct Geom {
     int bwd_rcap;       // home records a backward block stages at most (>= its threads)
 };
 
-constexpr int kBinChunk = 1024;        // most Gaussians per binning chunk (large frames)
-constexpr int kBinChunkMin = 256;      // fewest (more chunks when there are few frames)
 constexpr int kFrameBlockMaxT = 256;   // small frames: at most this many tiles
 constexpr int kFrameBlockMaxN = 16384; // and at most this many Gaussians
 constexpr int kClusterTiles = 16;            // frames up to this many tiles: one cluster per frame
@@ -69,9 +67,9 @@ constexpr int kClusterMaxBlocks = 4 * 148;   // ... while the launch has at most
 // weight is w = 2^{-(uhat_1^2 + uhat_2^2)} = exp(-q / 2).
 struct Workspace {
     int *err;       // device error word
-    int *done;      // [B] per-frame block counters of the tile scan (zero between launches)
     float4 *gr;     // [B*N][2]
-    int *hist;      // [B][nchunks][T]: chunk counts, then prefix over chunks
+    int *hist;      // [B][nslab][T]: slab counts, then exclusive prefix over slabs
+    int *tot;       // [B][T]: entries per tile
     int *offs;      // [B][T + 1]: absolute list start of every tile, frame end
     int *ids;       // [B][cap]: frame-local Gaussian ids, tile-major
 };
