@@ -41,13 +41,14 @@ pdr_status make_geom(int B, int N, int C, int H, int W, int k, Geom *g) {
     g->cap = (int)cap;
     // Binning slabs of 32 * R Gaussians (one scatter warp each): R = 8, halved
     // while the frames would give fewer than eight scatter warps per SM, but
-    // at least T / 128 so that the per-slab counts (B x slabs x T ints) stay
-    // within about four ints per Gaussian.  Slabs under 256 Gaussians divide
-    // 256 (R = 1, 2, 4).
+    // at least T / 64 so that the per-slab counts (B x slabs x T ints) stay
+    // within about two ints per Gaussian (measured on B200: 512-Gaussian slabs
+    // bin a 1024-tile frame faster than 256).  Slabs under 256 Gaussians
+    // divide 256 (R = 1, 2, 4).
     {
         int R = 8;
         while (R > 1 && (long long)B * ((N + 32 * R - 1) / (32 * R)) < 8 * 148) R >>= 1;
-        int rmin = (int)((T + 127) / 128);
+        int rmin = (int)((T + 63) / 64);
         if (rmin <= 8) rmin = rmin <= 1 ? 1 : rmin <= 2 ? 2 : rmin <= 4 ? 4 : 8;  // divides 256
         if (R < rmin) R = rmin;
         g->slab = 32 * R;

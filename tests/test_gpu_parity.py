@@ -318,18 +318,18 @@ def test_separate_bins_then_render_matches_one_call():
 @pytest.mark.parametrize("B,N,C,H,W,k", [
     (2, 40000, 1, 112, 144, 5),   # 64-Gaussian slabs, 625 per frame: the scan's runs exceed its registers
     (1, 70000, 1, 64, 64, 5),     # 32-Gaussian slabs (eight per count block), 2188 per frame, a ragged last one
-    (1, 20000, 2, 300, 240, 3),   # 285 tiles: 128-Gaussian slabs
-    (1, 3000, 1, 2048, 2048, 5),  # the most tiles a frame may have (16384): one 4096-Gaussian slab, 1-warp blocks
+    (1, 20000, 2, 300, 240, 3),   # 285 tiles: 256-Gaussian slabs, a ragged last one
+    (1, 3000, 1, 2048, 2048, 5),  # the most tiles a frame may have (16384): one 8192-Gaussian slab, 1-warp blocks
     (3, 1000, 2, 96, 160, 11),    # few frames, a ragged last slab
     (2, 4000, 1, 128, 128, 9),    # 125 slabs per frame, a ragged last block of warps
     (5, 333, 4, 32, 64, 9),       # 8 tiles, 11 slabs per frame
     (2, 30000, 2, 200, 328, 21),  # windows over up to 3 tiles per axis
-    (1, 5000, 3, 512, 768, 31),   # the largest window: 1536 tiles, 384-Gaussian slabs counted in two rounds
+    (1, 5000, 3, 512, 768, 31),   # the largest window: 1536 tiles, 768-Gaussian slabs counted in three rounds
 ])
 def test_slab_binning_paths(B, N, C, H, W, k):
     """Frames binned by the slab kernels (records and per-slab counts, the
     prefix over slabs per tile, the per-warp stable scatter): slabs of 32 to
-    4096 Gaussians, windows over 2 and 3 tiles per axis, ragged last slabs."""
+    8192 Gaussians, windows over 2 and 3 tiles per axis, ragged last slabs."""
     rng = np.random.default_rng(N + H)
     p = _edge_params(rng, B, N, C, H, W, k, smean=0.2, ssd=0.3)
     g = rng.standard_normal((B, C, H, W)).astype(np.float32)
