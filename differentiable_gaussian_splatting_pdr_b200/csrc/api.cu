@@ -260,8 +260,11 @@ pdr_status pdr_render_fwd_ex(const float *params, int B, int N, int C, int H, in
             cudaMemsetAsync(image, 0, esize * (size_t)g.B * g.C * g.H * g.W, s));
     }
     g.img_dtype = image_dtype;
-    g.out_vec2 = ((g.W & 1) == 0) && ((reinterpret_cast<uintptr_t>(image) & 7) == 0);
-    g.out_vec4 = ((g.W & 3) == 0) && ((reinterpret_cast<uintptr_t>(image) & 15) == 0);
+    // 2- and 4-pixel vector stores: rows of a multiple of 2 / 4 pixels and an
+    // image aligned to 2 / 4 elements.
+    const uintptr_t esz = image_dtype == PDR_F32 ? 4 : 2;
+    g.out_vec2 = ((g.W & 1) == 0) && ((reinterpret_cast<uintptr_t>(image) & (2 * esz - 1)) == 0);
+    g.out_vec4 = ((g.W & 3) == 0) && ((reinterpret_cast<uintptr_t>(image) & (4 * esz - 1)) == 0);
     if (!workspace_holds_bins && g.cluster_fwd && fwd_cluster_schedulable(g)) {
         // Small frames: bins + render in one clustered launch.
         st = from_cuda(clear_error_word(ws, s));
@@ -299,8 +302,10 @@ pdr_status pdr_render_bwd_ex(const float *params, const void *grad_image, int gr
     const Workspace ws = carve(workspace, L);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     g.img_dtype = grad_dtype;
-    g.stage_vec4 = grad_dtype == PDR_F32 && (g.W & 3) == 0 &&
-                   (reinterpret_cast<uintptr_t>(grad_image) & 15) == 0;
+    // Four consecutive dL/dI elements per vector load: rows of a multiple of 4
+    // elements and an image aligned to 4 elements (16 bytes fp32, 8 bytes half).
+    g.stage_vec4 = (g.W & 3) == 0 &&
+                   (reinterpret_cast<uintptr_t>(grad_image) & (grad_dtype == PDR_F32 ? 15 : 7)) == 0;
     if (!workspace_holds_fwd_bins) {
         st = from_cuda(bin(params, g, ws, s));
         if (st != PDR_OK) return st;

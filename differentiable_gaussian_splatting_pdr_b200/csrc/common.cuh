@@ -45,10 +45,10 @@ struct Geom {
     int frame_threads;  // threads of that block
     int cluster_fwd;    // 1: frames of <= kClusterTiles tiles, bins + forward in one launch
     int fwd_pl;         // forward pixels per lane (2 or 4)
-    int out_vec2;       // 1 if the output image allows 8-byte 2-pixel stores
-    int out_vec4;       // 1 if the output image allows 16-byte 4-pixel stores
+    int out_vec2;       // 1 if the output image allows 2-pixel vector stores
+    int out_vec4;       // 1 if the output image allows 4-pixel vector stores
     int img_dtype;      // storage of image / dL/dI: PDR_F32, PDR_F16 or PDR_BF16
-    int stage_vec4;     // 1: dL/dI is fp32, rows of a multiple of 4 floats, 16-byte aligned
+    int stage_vec4;     // 1: dL/dI rows of a multiple of 4 elements, image aligned to 4 elements
     int bwd_threads;    // threads per backward block
     int bwd_rcap;       // home records a backward block stages at most (>= its threads)
 };
@@ -149,6 +149,11 @@ __device__ __forceinline__ float img_load(const void *p, size_t i, int dtype) {
     if (dtype == 1) return __half2float(static_cast<const __half *>(p)[i]);
     if (dtype == 2) return __bfloat162float(static_cast<const __nv_bfloat16 *>(p)[i]);
     return static_cast<const float *>(p)[i];
+}
+// v rounded to nearest to fp16 (dtype 1) or bf16 (dtype 2), as raw bits.
+__device__ __forceinline__ unsigned short half_bits(float v, int dtype) {
+    return dtype == 1 ? __half_as_ushort(__float2half_rn(v))
+                      : __bfloat16_as_ushort(__float2bfloat16_rn(v));
 }
 __device__ __forceinline__ void img_store(void *p, size_t i, int dtype, float v) {
     if (dtype == 1)

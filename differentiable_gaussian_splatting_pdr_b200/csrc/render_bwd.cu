@@ -490,13 +490,13 @@ struct PairShape {
 };
 
 // Stages dL/dI of the pair kernels' region [X0 - r, X0 + 15 + r] x rows
-// [Y0 - r, Y0 + 15 + r] (zero outside it and outside the grid) for fp32
-// storage with rows of a multiple of 4 floats and a 16-byte aligned image:
-// thread (row, j) loads the aligned float4 of columns X0 - 8 + 4j .. + 3 of
-// every channel (one vector load each; guarded scalar loads where it
-// crosses the grid's edge) and writes the parity elements whose first pixel
-// it holds, the second pixel of a pair that ends past its float4 coming from
-// the next lane (the float4 to its right).
+// [Y0 - r, Y0 + 15 + r] (zero outside it and outside the grid) for rows of a
+// multiple of 4 elements and an image aligned to 4 elements: thread (row, j)
+// loads the aligned 4 elements of columns X0 - 8 + 4j .. + 3 of every channel
+// (one vector load each: a float4, or 8 bytes of fp16 / bf16 widened to fp32;
+// guarded scalar loads where it crosses the grid's edge) and writes the
+// parity elements whose first pixel it holds, the second pixel of a pair that
+// ends past its 4 elements coming from the next lane (the group to its right).
 template <int C, int K, int NT>
 __device__ __forceinline__ void stage_pairs_vec4(const void *__restrict__ gimg, const Geom &g,
                                                  int b, int X0, int Y0, float4 *halo4,
@@ -506,7 +506,6 @@ __device__ __forceinline__ void stage_pairs_vec4(const void *__restrict__ gimg, 
     constexpr int NJ = (8 + kTile + R + 1 + 3) / 4;  // float4 columns from X0 - 8
     static_assert(NJ == 8 && R <= 8, "one warp covers 4 rows of 8 float4 columns");
     constexpr int NCH = 2 * NP4 + NP2;
-    const float *img = static_cast<const float *>(gimg);
     for (int it0 = 0; it0 < S::ROWS * NJ; it0 += NT) {  // every lane runs every round (shuffle)
         const int it = it0 + (int)threadIdx.x;
         const int row = it / NJ, j = it - row * NJ;
@@ -518,14 +517,24 @@ __device__ __forceinline__ void stage_pairs_vec4(const void *__restrict__ gimg, 
         for (int c = 0; c < NCH; ++c) {
             v[c][0] = v[c][1] = v[c][2] = v[c][3] = 0.0f;
             if (c < C && rowin) {
-                const float *src = img + (((size_t)b * C + c) * g.H + y) * g.W;
+                const size_t row0 = (((size_t)b * C + c) * g.H + y) * g.W;
                 if (x4 >= 0 && x4 + 3 < g.W) {
-                    const float4 q = *reinterpret_cast<const float4 *>(src + x4);
-                    v[c][0] = q.x; v[c][1] = q.y; v[c][2] = q.z; v[c][3] = q.w;
+                    if (g.img_dtype == 0) {  // fp32
+                        const float4 q = *reinterpret_cast<const float4 *>(static_cast<const float *>(gimg) + row0 + x4);
+                        v[c][0] = q.x; v[c][1] = q.y; v[c][2] = q.z; v[c][3] = q.w;
+                    } else {
+                        const uint2 q = *reinterpret_cast<const uint2 *>(static_cast<const unsigned short *>(gimg) + row0 + x4);
+                        const unsigned hw[4] = {q.x & 0xffffu, q.x >> 16, q.y & 0xffffu, q.y >> 16};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            v[c][e] = g.img_dtype == 1  // fp16, else bf16
+                                          ? __half2float(__ushort_as_half((unsigned short)hw[e]))
+                                          : __bfloat162float(__ushort_as_bfloat16((unsigned short)hw[e]));
+                    }
                 } else {
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
-                        if (x4 + e >= 0 && x4 + e < g.W) v[c][e] = src[x4 + e];
+                        if (x4 + e >= 0 && x4 + e < g.W) v[c][e] = img_load(gimg, row0 + x4 + e, g.img_dtype);
                 }
             }
             // zero outside [X0 - r, X0 + 15 + r]

@@ -195,12 +195,25 @@ __device__ __forceinline__ void store_tile(const Geom &g, int b, int X0, int Y0,
     const int x = X0 + 4 * (grp & 3) + lcol, y = Y0 + 4 * (grp >> 2) + lrow;
     if (y >= g.H) return;
     if (g.img_dtype != 0) {  // fp16 / bf16 storage: fp32 sums, rounded to nearest once
+        const bool hvec = (x + PL - 1 < g.W) && (PL == 4 ? g.out_vec4 : g.out_vec2);
 #pragma unroll
         for (int c = 0; c < C; ++c) {
             const size_t o = (((size_t)b * C + c) * g.H + y) * g.W + x;
+            if (hvec) {
+                unsigned short hb[PL];
 #pragma unroll
-            for (int j = 0; j < PL; ++j)
-                if (x + j < g.W) img_store(image_, o + j, g.img_dtype, acc[j][c]);
+                for (int j = 0; j < PL; ++j) hb[j] = half_bits(acc[j][c], g.img_dtype);
+                unsigned short *dst = static_cast<unsigned short *>(image_) + o;
+                if constexpr (PL == 4)
+                    *reinterpret_cast<uint2 *>(dst) = make_uint2(hb[0] | ((unsigned)hb[1] << 16),
+                                                                 hb[2] | ((unsigned)hb[3] << 16));
+                else
+                    *reinterpret_cast<unsigned *>(dst) = hb[0] | ((unsigned)hb[1] << 16);
+            } else {
+#pragma unroll
+                for (int j = 0; j < PL; ++j)
+                    if (x + j < g.W) img_store(image_, o + j, g.img_dtype, acc[j][c]);
+            }
         }
         return;
     }
