@@ -178,6 +178,20 @@ def test_long_lists_in_one_tile():
     check_all(p, g, H, W, k)
 
 
+@pytest.mark.parametrize("W", [32, 30])
+def test_long_lists_pixel_pair_backward(W):
+    """Thousands of home Gaussians in one tile with k = 15: more than the pixel-pair
+    backward's record area holds, so the block runs several record rounds; W = 32
+    stages dL/dI with vector loads, W = 30 element by element."""
+    rng = np.random.default_rng(9 + W)
+    B, N, C, H, k = 2, 3000, 3, 32, 15
+    p = _edge_params(rng, B, N, C, H, W, k)
+    p[..., 0] = rng.uniform(3, 12, (B, N))
+    p[..., 1] = rng.uniform(3, 12, (B, N))
+    g = rng.standard_normal((B, C, H, W)).astype(np.float32)
+    check_all(p, g, H, W, k)
+
+
 def test_autograd_matches_direct_calls():
     w = WORKLOADS["mono64"].scaled(B=3)
     p, g = make_inputs(w)
