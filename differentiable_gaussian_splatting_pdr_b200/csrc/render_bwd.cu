@@ -497,7 +497,7 @@ struct PairShape {
 // guarded scalar loads where it crosses the grid's edge) and writes the
 // parity elements whose first pixel it holds, the second pixel of a pair that
 // ends past its 4 elements coming from the next lane (the group to its right).
-template <int C, int K, int NT>
+template <int C, int K, int NT, bool HALF>
 __device__ __forceinline__ void stage_pairs_vec4(const void *__restrict__ gimg, const Geom &g,
                                                  int b, int X0, int Y0, float4 *halo4,
                                                  float2 *halo2) {
@@ -519,7 +519,7 @@ __device__ __forceinline__ void stage_pairs_vec4(const void *__restrict__ gimg, 
             if (c < C && rowin) {
                 const size_t row0 = (((size_t)b * C + c) * g.H + y) * g.W;
                 if (x4 >= 0 && x4 + 3 < g.W) {
-                    if (g.img_dtype == 0) {  // fp32
+                    if constexpr (!HALF) {
                         const float4 q = *reinterpret_cast<const float4 *>(static_cast<const float *>(gimg) + row0 + x4);
                         v[c][0] = q.x; v[c][1] = q.y; v[c][2] = q.z; v[c][3] = q.w;
                     } else {
@@ -617,7 +617,10 @@ __global__ void __launch_bounds__(NT, 896 / NT) k_bwd_pairs(const float *__restr
     load_pass<NT, kPer>(ids, L0, L1, raw, valid);
 
     if (g.stage_vec4) {
-        stage_pairs_vec4<C, K, NT>(gimg, g, b, X0, Y0, halo4, halo2);
+        if (g.img_dtype == 0)
+            stage_pairs_vec4<C, K, NT, false>(gimg, g, b, X0, Y0, halo4, halo2);
+        else
+            stage_pairs_vec4<C, K, NT, true>(gimg, g, b, X0, Y0, halo4, halo2);
     } else {
         // Stage dL/dI over [X0 - r, X0 + 15 + r]^2 (zero outside the grid; the
         // column after it, read only as the masked pixel of a last pair, is zero
