@@ -366,7 +366,7 @@ __global__ void __launch_bounds__(32 * kSlabWarps) k_slab_scatter(
 // Warp w owns the contiguous slab [w * S, (w + 1) * S) of the frame's
 // Gaussians: it computes their records and counts them per tile; one block
 // scan turns the per-tile totals into the tiles' list starts; then every
-// warp scatters its slab as in k_scatter.
+// warp scatters its slab with the lane-mask ranks described above.
 __global__ void __launch_bounds__(1024) k_bin_frame(const float *__restrict__ params, Geom g,
                                                     float4 *__restrict__ gr,
                                                     int *__restrict__ offs,
