@@ -19,9 +19,16 @@
 // block per frame, does the records, the counts, the tile offsets and the
 // stable scatter in shared memory (ranks from a per-tile prefix over the
 // block's warps).  Same lists, same order.
+#include <cooperative_groups.h>
+#include <map>
+#include <mutex>
+#include <tuple>
+
 #include "common.cuh"
 
 namespace pdr {
+
+namespace cg = cooperative_groups;
 
 namespace {
 
@@ -439,6 +446,116 @@ __global__ void __launch_bounds__(1024) k_bin_frame(const float *__restrict__ pa
               tbase, ids, err);
 }
 
+// Frames of at most kClusterTiles tiles: one thread-block cluster per frame
+// (grid (T, B), cluster (T, 1, 1)), block q owning tile q and the q-th chunk of
+// the frame's Gaussians.  Each block computes its chunk's records and counts
+// them per tile; the counts of all blocks are read through distributed shared
+// memory, giving the tiles' list starts and this chunk's first slot in every
+// tile (the counts of the chunks before it); the chunk is then scattered in
+// rounds of kClusterBinThreads with the per-warp lane-mask ranks.  One launch,
+// no counts in global memory.
+constexpr int kClusterBinThreads = 256;
+
+__global__ void __launch_bounds__(kClusterBinThreads) k_bin_cluster(
+    const float *__restrict__ params, Geom g, float4 *__restrict__ gr, int *__restrict__ offs,
+    int *__restrict__ ids, int *__restrict__ err) {
+    constexpr int NW = kClusterBinThreads / 32;
+    __shared__ int cnt[kClusterTiles];                    // this chunk's count per tile
+    __shared__ int tab[kClusterTiles][kClusterTiles];     // tab[r][t]: chunk r's count in tile t
+    __shared__ int tstart[kClusterTiles + 1];             // frame-relative list start per tile
+    __shared__ int base[kClusterTiles];                   // next slot of this chunk per tile
+    __shared__ unsigned masks[NW][kClusterTiles];         // per-warp lane masks of a round
+    cg::cluster_group cluster = cg::this_cluster();
+    const int T = g.T;
+    const int q = (int)cluster.block_rank();
+    const int b = blockIdx.y;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const unsigned lt = lanemask_lt();
+    if (tid < kClusterTiles) cnt[tid] = 0;
+    if (tid < NW * kClusterTiles) masks[tid / kClusterTiles][tid % kClusterTiles] = 0u;
+    __syncthreads();
+    const int chunk = (g.N + T - 1) / T;
+    const int i0 = min(q * chunk, g.N), i1 = min(i0 + chunk, g.N);
+    for (int i = i0 + tid; i < i1; i += kClusterBinThreads) {
+        const size_t gid = (size_t)b * g.N + i;
+        float4 A, Q;
+        gaussian_record(params + gid * g.P, A, Q);
+        gr[2 * gid] = A;
+        gr[2 * gid + 1] = Q;
+        int tx0, ty0, nx, ny;
+        window_tiles(__float_as_int(Q.z), __float_as_int(Q.w), g, tx0, ty0, nx, ny);
+        for (int dy = 0; dy < ny; ++dy)
+            for (int dx = 0; dx < nx; ++dx) atomicAdd(&cnt[(ty0 + dy) * g.TX + tx0 + dx], 1);
+    }
+    cluster.sync();  // every chunk's counts are final
+    for (int j = tid; j < T * T; j += kClusterBinThreads) {
+        const int r = j / T, tt = j - r * T;
+        tab[r][tt] = *cluster.map_shared_rank(cnt + tt, r);
+    }
+    cluster.sync();  // no block leaves (or reuses cnt) while a peer may still read it
+    if (warp == 0) {  // lane tt sums tile tt's column, then a warp scan over the tiles
+        int col = 0, below = 0;
+        if (lane < T) {
+            for (int r = 0; r < T; ++r) {
+                const int v = tab[r][lane];
+                col += v;
+                below += r < q ? v : 0;
+            }
+        }
+        int incl = col;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int u = __shfl_up_sync(0xffffffffu, incl, d);
+            if (lane >= d) incl += u;
+        }
+        if (lane < T) {
+            tstart[lane] = incl - col;
+            base[lane] = incl - col + below;
+        }
+        if (lane == T - 1) tstart[T] = incl;
+    }
+    __syncthreads();
+    const int frame0 = b * g.cap;
+    if (q == 0)
+        for (int tt = tid; tt <= T; tt += kClusterBinThreads)
+            offs[(size_t)b * (T + 1) + tt] = frame0 + tstart[tt];
+    const int lo = frame0, hi = frame0 + g.cap;
+    for (int s0 = i0; s0 < i1; s0 += kClusterBinThreads) {  // block-uniform rounds
+        const int i = s0 + tid;
+        int tx0 = 0, ty0 = 0, nx = 0, ny = 0, ht = -1;
+        if (i < i1) {
+            const float4 Q = gr[2 * ((size_t)b * g.N + i) + 1];
+            const int cx = __float_as_int(Q.z), cy = __float_as_int(Q.w);
+            window_tiles(cx, cy, g, tx0, ty0, nx, ny);
+            if (nx) ht = home_tile(cx, cy, g);
+        }
+        for (int dy = 0; dy < ny; ++dy)
+            for (int dx = 0; dx < nx; ++dx)
+                atomicOr(&masks[warp][(ty0 + dy) * g.TX + tx0 + dx], 1u << lane);
+        __syncthreads();
+        for (int dy = 0; dy < ny; ++dy)
+            for (int dx = 0; dx < nx; ++dx) {
+                const int tt = (ty0 + dy) * g.TX + tx0 + dx;
+                int pre = base[tt] + __popc(masks[warp][tt] & lt);
+                for (int w = 0; w < warp; ++w) pre += __popc(masks[w][tt]);
+                const int slot = frame0 + pre;
+                if (slot >= lo && slot < hi)
+                    ids[slot] = (int)((unsigned)i | (tt == ht ? kHomeFlag : 0u));
+                else
+                    atomicOr(err, kErrListBounds);
+            }
+        __syncthreads();
+        if (tid < T) {
+            int add = 0;
+            for (int w = 0; w < NW; ++w) add += __popc(masks[w][tid]);
+            base[tid] += add;
+        }
+        __syncthreads();
+        if (tid < NW * kClusterTiles) masks[tid / kClusterTiles][tid % kClusterTiles] = 0u;
+        __syncthreads();
+    }
+}
+
 __global__ void k_copy_ids(int *__restrict__ dst, const int *__restrict__ src, size_t n) {
     for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
          i += (size_t)gridDim.x * blockDim.x)
@@ -481,9 +598,65 @@ static cudaError_t allow_smem(K kernel, size_t bytes) {
     return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
+// The clustered binner for these sizes can be scheduled on the current device
+// (at least one cluster of T blocks fits); cached per device and T.
+static bool bin_cluster_fits(const Geom &g) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    static std::mutex mu;
+    static std::map<std::pair<int, int>, bool> known;
+    std::lock_guard<std::mutex> lock(mu);
+    const auto key = std::make_pair(dev, g.T);
+    const auto it = known.find(key);
+    if (it != known.end()) return it->second;
+    bool ok = true;
+    if (g.T > 8 && cudaFuncSetAttribute(k_bin_cluster, cudaFuncAttributeNonPortableClusterSizeAllowed,
+                                        1) != cudaSuccess) {
+        cudaGetLastError();
+        ok = false;
+    }
+    if (ok) {
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        cfg.gridDim = dim3(g.T, 1, 1);
+        cfg.blockDim = dim3(kClusterBinThreads, 1, 1);
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = g.T;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, k_bin_cluster, &cfg) != cudaSuccess) {
+            cudaGetLastError();
+            n = 0;
+        }
+        ok = n > 0;
+    }
+    known[key] = ok;
+    return ok;
+}
+
 cudaError_t launch_bin(const float *params, const Geom &g, const Workspace &ws,
                        cudaStream_t s) {
     cudaError_t e;
+    if (g.T <= kClusterTiles && bin_cluster_fits(g)) {
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        cfg.gridDim = dim3(g.T, g.B, 1);
+        cfg.blockDim = dim3(kClusterBinThreads, 1, 1);
+        cfg.dynamicSmemBytes = 0;
+        cfg.stream = s;
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = g.T;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, k_bin_cluster, params, g, ws.gr, ws.offs, ws.ids, ws.err);
+        if (e != cudaSuccess) return e;
+        return cudaGetLastError();
+    }
     if (g.frame_block) {
         const size_t sf = bin_frame_smem(g);
         if ((e = allow_smem(k_bin_frame, sf)) != cudaSuccess) return e;
