@@ -15,8 +15,10 @@
 //   k_slab_scatter  per block: the tiles' list starts (block scan of the
 //                   totals); per slab: stable ranks in rounds of 32 from
 //                   lane masks, written at start + slab prefix + rank.
-// Small frames (g.frame_block) take one launch instead: k_bin_frame, one
-// block per frame, does the records, the counts, the tile offsets and the
+// Frames of at most 16 tiles take one launch instead: k_bin_cluster, one
+// thread-block cluster per frame (chunk counts exchanged through distributed
+// shared memory).  Other small frames (g.frame_block) take k_bin_frame, one
+// block per frame doing the records, the counts, the tile offsets and the
 // stable scatter in shared memory (ranks from a per-tile prefix over the
 // block's warps).  Same lists, same order.
 #include <cooperative_groups.h>

@@ -353,16 +353,33 @@ def test_slab_binning_paths(B, N, C, H, W, k):
 @pytest.mark.parametrize("B,N,C,H,W,k", [
     (3, 1000, 2, 96, 160, 11),   # 60 tiles
     (2, 4000, 1, 128, 128, 9),   # 64 tiles, 4000 ids
-    (5, 333, 4, 32, 64, 9),      # 8 tiles, a ragged last warp of ids
-    (2, 5000, 3, 48, 80, 7),     # 15 tiles, 5000 ids
+    (5, 333, 4, 32, 64, 9),      # 8 tiles: the clustered binner
+    (2, 5000, 3, 48, 80, 7),     # 15 tiles: the clustered binner, 5000 ids
     (1, 980, 1, 192, 256, 5),    # 192 tiles, 16-warp frame blocks
 ])
 def test_frame_block_binning(B, N, C, H, W, k):
-    """Frames binned by one block each (up to 256 tiles; used when there are at
-    least as many frames as SMs, so B becomes 150 here), windows partly and
-    wholly off the grid, ragged last warp of ids."""
+    """Many frames (B becomes 150 here, at least one frame per SM): frames of 17
+    to 256 tiles are binned by one block each, frames of at most 16 tiles by one
+    thread-block cluster each; windows partly and wholly off the grid, ragged
+    last warp of ids."""
     B = 150
     rng = np.random.default_rng(B * 7 + N + W)
+    p = _edge_params(rng, B, N, C, H, W, k)
+    g = rng.standard_normal((B, C, H, W)).astype(np.float32)
+    check_all(p, g, H, W, k)
+
+
+@pytest.mark.parametrize("B,N,C,H,W,k", [
+    (1, 300, 2, 16, 16, 9),      # one tile: a cluster of one block
+    (4, 5000, 1, 64, 64, 9),     # 16 tiles: the largest (non-portable) cluster
+    (3, 7, 3, 40, 56, 15),       # fewer Gaussians than tiles: empty chunks
+    (2, 2501, 4, 33, 47, 7),     # ragged tiles, a chunk size not dividing N
+    (2, 3000, 1, 48, 48, 31),    # windows over 3 tiles per axis
+])
+def test_cluster_binning(B, N, C, H, W, k):
+    """Frames of at most 16 tiles, binned by one thread-block cluster each
+    (chunk counts exchanged through distributed shared memory)."""
+    rng = np.random.default_rng(B * 13 + N + W)
     p = _edge_params(rng, B, N, C, H, W, k)
     g = rng.standard_normal((B, C, H, W)).astype(np.float32)
     check_all(p, g, H, W, k)
