@@ -15,7 +15,7 @@
 //   k_slab_scatter  per block: the tiles' list starts (block scan of the
 //                   totals); per slab: stable ranks in rounds of 32 from
 //                   lane masks, written at start + slab prefix + rank.
-// Frames of at most 16 tiles take one launch instead: k_bin_cluster, one
+// Frames of at most 64 tiles take one launch instead: k_bin_cluster, one
 // thread-block cluster per frame (chunk counts exchanged through distributed
 // shared memory).  Other small frames (g.frame_block) take k_bin_frame, one
 // block per frame doing the records, the counts, the tile offsets and the
@@ -448,35 +448,39 @@ __global__ void __launch_bounds__(1024) k_bin_frame(const float *__restrict__ pa
               tbase, ids, err);
 }
 
-// Frames of at most kClusterTiles tiles: one thread-block cluster per frame
-// (grid (T, B), cluster (T, 1, 1)), block q owning tile q and the q-th chunk of
-// the frame's Gaussians.  Each block computes its chunk's records and counts
-// them per tile; the counts of all blocks are read through distributed shared
-// memory, giving the tiles' list starts and this chunk's first slot in every
-// tile (the counts of the chunks before it); the chunk is then scattered in
-// rounds of kClusterBinThreads with the per-warp lane-mask ranks.  One launch,
-// no counts in global memory.
+// Frames of at most kClusterBinMaxT tiles: one thread-block cluster of CS =
+// min(T, 16) blocks per frame (grid (CS, B), cluster (CS, 1, 1)), block q
+// owning the q-th chunk of the frame's Gaussians.  Each block computes its
+// chunk's records and counts them per tile; the counts of all blocks are read
+// through distributed shared memory, giving the tiles' list starts and this
+// chunk's first slot in every tile (the counts of the chunks before it); the
+// chunk is then scattered in rounds of kClusterBinThreads with the per-warp
+// lane-mask ranks.  One launch, no counts in global memory.
 constexpr int kClusterBinThreads = 256;
+constexpr int kClusterBinMaxT = 64;    // most tiles per frame
+constexpr int kClusterBinMaxCS = 16;   // most blocks per cluster (non-portable above 8)
+
+__host__ __device__ constexpr int bin_cluster_size(int T) { return T < kClusterBinMaxCS ? T : kClusterBinMaxCS; }
 
 __global__ void __launch_bounds__(kClusterBinThreads) k_bin_cluster(
     const float *__restrict__ params, Geom g, float4 *__restrict__ gr, int *__restrict__ offs,
     int *__restrict__ ids, int *__restrict__ err) {
-    constexpr int NW = kClusterBinThreads / 32;
-    __shared__ int cnt[kClusterTiles];                    // this chunk's count per tile
-    __shared__ int tab[kClusterTiles][kClusterTiles];     // tab[r][t]: chunk r's count in tile t
-    __shared__ int tstart[kClusterTiles + 1];             // frame-relative list start per tile
-    __shared__ int base[kClusterTiles];                   // next slot of this chunk per tile
-    __shared__ unsigned masks[NW][kClusterTiles];         // per-warp lane masks of a round
+    constexpr int NW = kClusterBinThreads / 32, MT = kClusterBinMaxT;
+    __shared__ int cnt[MT];                          // this chunk's count per tile
+    __shared__ int tab[kClusterBinMaxCS][MT];        // tab[r][t]: chunk r's count in tile t
+    __shared__ int tstart[MT + 1];                   // frame-relative list start per tile
+    __shared__ int base[MT];                         // next slot of this chunk per tile
+    __shared__ unsigned masks[NW][MT];               // per-warp lane masks of a round
     cg::cluster_group cluster = cg::this_cluster();
-    const int T = g.T;
+    const int T = g.T, CS = bin_cluster_size(T);
     const int q = (int)cluster.block_rank();
     const int b = blockIdx.y;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const unsigned lt = lanemask_lt();
-    if (tid < kClusterTiles) cnt[tid] = 0;
-    if (tid < NW * kClusterTiles) masks[tid / kClusterTiles][tid % kClusterTiles] = 0u;
+    for (int t = tid; t < MT; t += kClusterBinThreads) cnt[t] = 0;
+    for (int t = tid; t < NW * MT; t += kClusterBinThreads) masks[t / MT][t % MT] = 0u;
     __syncthreads();
-    const int chunk = (g.N + T - 1) / T;
+    const int chunk = (g.N + CS - 1) / CS;
     const int i0 = min(q * chunk, g.N), i1 = min(i0 + chunk, g.N);
     for (int i = i0 + tid; i < i1; i += kClusterBinThreads) {
         const size_t gid = (size_t)b * g.N + i;
@@ -490,31 +494,42 @@ __global__ void __launch_bounds__(kClusterBinThreads) k_bin_cluster(
             for (int dx = 0; dx < nx; ++dx) atomicAdd(&cnt[(ty0 + dy) * g.TX + tx0 + dx], 1);
     }
     cluster.sync();  // every chunk's counts are final
-    for (int j = tid; j < T * T; j += kClusterBinThreads) {
+    for (int j = tid; j < CS * T; j += kClusterBinThreads) {
         const int r = j / T, tt = j - r * T;
         tab[r][tt] = *cluster.map_shared_rank(cnt + tt, r);
     }
-    cluster.sync();  // no block leaves (or reuses cnt) while a peer may still read it
-    if (warp == 0) {  // lane tt sums tile tt's column, then a warp scan over the tiles
-        int col = 0, below = 0;
-        if (lane < T) {
-            for (int r = 0; r < T; ++r) {
-                const int v = tab[r][lane];
-                col += v;
-                below += r < q ? v : 0;
-            }
+    cluster.sync();  // no block leaves while a peer may still read its counts
+    if (warp == 0) {
+        // Lane l takes tiles 2l and 2l + 1: their totals and the counts of the
+        // chunks before this one; one warp scan over the pairs.
+        int col[2] = {0, 0}, below[2] = {0, 0};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int tt = 2 * lane + h;
+            if (tt < T)
+                for (int r = 0; r < CS; ++r) {
+                    const int v = tab[r][tt];
+                    col[h] += v;
+                    below[h] += r < q ? v : 0;
+                }
         }
-        int incl = col;
+        const int pair = col[0] + col[1];
+        int incl = pair;
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
             const int u = __shfl_up_sync(0xffffffffu, incl, d);
             if (lane >= d) incl += u;
         }
-        if (lane < T) {
-            tstart[lane] = incl - col;
-            base[lane] = incl - col + below;
+        const int ex0 = incl - pair, ex1 = ex0 + col[0];
+        if (2 * lane < T) {
+            tstart[2 * lane] = ex0;
+            base[2 * lane] = ex0 + below[0];
         }
-        if (lane == T - 1) tstart[T] = incl;
+        if (2 * lane + 1 < T) {
+            tstart[2 * lane + 1] = ex1;
+            base[2 * lane + 1] = ex1 + below[1];
+        }
+        if (lane == 31) tstart[T] = incl;
     }
     __syncthreads();
     const int frame0 = b * g.cap;
@@ -547,13 +562,13 @@ __global__ void __launch_bounds__(kClusterBinThreads) k_bin_cluster(
                     atomicOr(err, kErrListBounds);
             }
         __syncthreads();
-        if (tid < T) {
+        for (int t = tid; t < T; t += kClusterBinThreads) {
             int add = 0;
-            for (int w = 0; w < NW; ++w) add += __popc(masks[w][tid]);
-            base[tid] += add;
+            for (int w = 0; w < NW; ++w) add += __popc(masks[w][t]);
+            base[t] += add;
         }
         __syncthreads();
-        if (tid < NW * kClusterTiles) masks[tid / kClusterTiles][tid % kClusterTiles] = 0u;
+        for (int t = tid; t < NW * MT; t += kClusterBinThreads) masks[t / MT][t % MT] = 0u;
         __syncthreads();
     }
 }
@@ -601,7 +616,7 @@ static cudaError_t allow_smem(K kernel, size_t bytes) {
 }
 
 // The clustered binner for these sizes can be scheduled on the current device
-// (at least one cluster of T blocks fits); cached per device and T.
+// (at least one cluster of min(T, 16) blocks fits); cached per device and T.
 static bool bin_cluster_fits(const Geom &g) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) return false;
@@ -612,18 +627,19 @@ static bool bin_cluster_fits(const Geom &g) {
     const auto it = known.find(key);
     if (it != known.end()) return it->second;
     bool ok = true;
-    if (g.T > 8 && cudaFuncSetAttribute(k_bin_cluster, cudaFuncAttributeNonPortableClusterSizeAllowed,
-                                        1) != cudaSuccess) {
+    const int CS = bin_cluster_size(g.T);
+    if (CS > 8 && cudaFuncSetAttribute(k_bin_cluster, cudaFuncAttributeNonPortableClusterSizeAllowed,
+                                       1) != cudaSuccess) {
         cudaGetLastError();
         ok = false;
     }
     if (ok) {
         cudaLaunchConfig_t cfg = {};
         cudaLaunchAttribute attr[1];
-        cfg.gridDim = dim3(g.T, 1, 1);
+        cfg.gridDim = dim3(CS, 1, 1);
         cfg.blockDim = dim3(kClusterBinThreads, 1, 1);
         attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = g.T;
+        attr[0].val.clusterDim.x = CS;
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = 1;
         cfg.attrs = attr;
@@ -642,15 +658,16 @@ static bool bin_cluster_fits(const Geom &g) {
 cudaError_t launch_bin(const float *params, const Geom &g, const Workspace &ws,
                        cudaStream_t s) {
     cudaError_t e;
-    if (g.T <= kClusterTiles && bin_cluster_fits(g)) {
+    if (g.T <= kClusterBinMaxT && bin_cluster_fits(g)) {
+        const int CS = bin_cluster_size(g.T);
         cudaLaunchConfig_t cfg = {};
         cudaLaunchAttribute attr[1];
-        cfg.gridDim = dim3(g.T, g.B, 1);
+        cfg.gridDim = dim3(CS, g.B, 1);
         cfg.blockDim = dim3(kClusterBinThreads, 1, 1);
         cfg.dynamicSmemBytes = 0;
         cfg.stream = s;
         attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = g.T;
+        attr[0].val.clusterDim.x = CS;
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = 1;
         cfg.attrs = attr;

@@ -330,20 +330,19 @@ def test_separate_bins_then_render_matches_one_call():
 
 
 @pytest.mark.parametrize("B,N,C,H,W,k", [
-    (2, 40000, 1, 112, 144, 5),   # 64-Gaussian slabs, 625 per frame: the scan's runs exceed its registers
-    (1, 70000, 1, 64, 64, 5),     # 32-Gaussian slabs (eight per count block), 2188 per frame, a ragged last one
+    (1, 100000, 1, 160, 160, 5),  # 100 tiles, 64-Gaussian slabs, 1563 per frame: the scan's runs exceed its registers
+    (2, 20000, 2, 200, 240, 3),   # 195 tiles: 128-Gaussian slabs, a ragged last one
     (1, 20000, 2, 300, 240, 3),   # 285 tiles: 256-Gaussian slabs, a ragged last one
     (1, 3000, 1, 2048, 2048, 5),  # the most tiles a frame may have (16384): one 8192-Gaussian slab, 1-warp blocks
-    (3, 1000, 2, 96, 160, 11),    # few frames, a ragged last slab
-    (2, 4000, 1, 128, 128, 9),    # 125 slabs per frame, a ragged last block of warps
-    (5, 333, 4, 32, 64, 9),       # 8 tiles, 11 slabs per frame
+    (3, 1000, 2, 96, 176, 11),    # 66 tiles, few Gaussians
     (2, 30000, 2, 200, 328, 21),  # windows over up to 3 tiles per axis
     (1, 5000, 3, 512, 768, 31),   # the largest window: 1536 tiles, 768-Gaussian slabs counted in three rounds
 ])
 def test_slab_binning_paths(B, N, C, H, W, k):
-    """Frames binned by the slab kernels (records and per-slab counts, the
-    prefix over slabs per tile, the per-warp stable scatter): slabs of 32 to
-    8192 Gaussians, windows over 2 and 3 tiles per axis, ragged last slabs."""
+    """Frames of more than 64 tiles, binned by the slab kernels (records and
+    per-slab counts, the prefix over slabs per tile, the per-warp stable
+    scatter): slabs of 64 to 8192 Gaussians, windows over 2 and 3 tiles per
+    axis, ragged last slabs."""
     rng = np.random.default_rng(N + H)
     p = _edge_params(rng, B, N, C, H, W, k, smean=0.2, ssd=0.3)
     g = rng.standard_normal((B, C, H, W)).astype(np.float32)
@@ -351,15 +350,15 @@ def test_slab_binning_paths(B, N, C, H, W, k):
 
 
 @pytest.mark.parametrize("B,N,C,H,W,k", [
-    (3, 1000, 2, 96, 160, 11),   # 60 tiles
-    (2, 4000, 1, 128, 128, 9),   # 64 tiles, 4000 ids
+    (3, 1000, 2, 96, 176, 11),   # 66 tiles, a frame block
+    (2, 4000, 1, 144, 128, 9),   # 72 tiles, 4000 ids
     (5, 333, 4, 32, 64, 9),      # 8 tiles: the clustered binner
     (2, 5000, 3, 48, 80, 7),     # 15 tiles: the clustered binner, 5000 ids
     (1, 980, 1, 192, 256, 5),    # 192 tiles, 16-warp frame blocks
 ])
 def test_frame_block_binning(B, N, C, H, W, k):
-    """Many frames (B becomes 150 here, at least one frame per SM): frames of 17
-    to 256 tiles are binned by one block each, frames of at most 16 tiles by one
+    """Many frames (B becomes 150 here, at least one frame per SM): frames of 65
+    to 256 tiles are binned by one block each, frames of at most 64 tiles by one
     thread-block cluster each; windows partly and wholly off the grid, ragged
     last warp of ids."""
     B = 150
@@ -371,14 +370,18 @@ def test_frame_block_binning(B, N, C, H, W, k):
 
 @pytest.mark.parametrize("B,N,C,H,W,k", [
     (1, 300, 2, 16, 16, 9),      # one tile: a cluster of one block
-    (4, 5000, 1, 64, 64, 9),     # 16 tiles: the largest (non-portable) cluster
-    (3, 7, 3, 40, 56, 15),       # fewer Gaussians than tiles: empty chunks
+    (4, 5000, 1, 64, 64, 9),     # 16 tiles: 16 blocks, the largest (non-portable) cluster
+    (3, 7, 3, 40, 56, 15),       # fewer Gaussians than blocks: empty chunks
     (2, 2501, 4, 33, 47, 7),     # ragged tiles, a chunk size not dividing N
     (2, 3000, 1, 48, 48, 31),    # windows over 3 tiles per axis
+    (2, 3000, 3, 64, 128, 11),   # 32 tiles in 16 blocks
+    (1, 70000, 1, 64, 64, 5),    # 4375 Gaussians per block: many scatter rounds
+    (1, 500, 2, 100, 100, 9),    # 49 tiles, ragged both ways
+    (3, 20, 1, 128, 128, 5),     # 64 tiles, the most the clustered binner takes; few Gaussians
 ])
 def test_cluster_binning(B, N, C, H, W, k):
-    """Frames of at most 16 tiles, binned by one thread-block cluster each
-    (chunk counts exchanged through distributed shared memory)."""
+    """Frames of at most 64 tiles, binned by one thread-block cluster of up to 16
+    blocks each (chunk counts exchanged through distributed shared memory)."""
     rng = np.random.default_rng(B * 13 + N + W)
     p = _edge_params(rng, B, N, C, H, W, k)
     g = rng.standard_normal((B, C, H, W)).astype(np.float32)
