@@ -445,20 +445,27 @@ __global__ void __launch_bounds__(NT, C > 4 ? 1 : 1024 / NT) k_bwd(const float *
 // decomposition and the same seven sums per Gaussian as k_bwd, but every
 // lane works on two horizontally adjacent pixels at once with the packed
 // f32x2 arithmetic of sm_100 (one instruction issues two FP32 FMAs), which
-// halves the issue slots of the inner loop; the loop is then bound by the
-// FMA pipe itself.
+// halves the issue slots of the inner loop.
 //
-// A window row of k pixels (k odd) is covered by (k + 1) / 2 pairs whose
-// last pixel lies just outside the window and is masked (its weight is
-// 2^-inf = 0).  So that every window starts on a pair boundary whatever its
-// parity, dL/dI is staged twice: pairs starting at even x and pairs starting
-// at odd x.  Two channels of a pair share one float4 (c lo, c hi, c+1 lo,
-// c+1 hi) and an odd last channel has a float2 plane of its own, so one
-// vector load per two channels yields the packed operands directly.  The
-// pair slots of a window (rows x pairs, row-major) are dealt to the 8 lanes
-// of a group in turn: lane l takes pair column l % NPW of rows l / NPW,
-// l / NPW + RPS, ...  Staged rows have a pitch congruent to the pairs per row
-// modulo 8, so the 8 lanes of a group always read 8 consecutive elements.
+// A window row of k pixels (k odd) is covered by (k + 1) / 2 pairs, one of
+// whose pixels lies just outside the window and is masked (its weight is
+// 2^-inf = 0).  dL/dI is staged once, in pairs that start at even x: a window
+// that starts at even x takes its pairs from its first pixel and masks the
+// pixel after its last; one that starts at odd x takes them from the pixel
+// before its first, which it masks.  Two channels of a pair share one float4
+// (c lo, c hi, c+1 lo, c+1 hi) and an odd last channel has a float2 plane of
+// its own, so one vector load per two channels yields the packed operands
+// directly.  Lane l of a group takes pair column l of every window row
+// (k = 13 leaves lane 7 idle).
+//
+// Per lane, the sums are formed from three row moments of its column: with
+// jc = row - r and U = uhat at the column's pixel of the window's centre row,
+// uhat = U + jc (beta_1, beta_2) along the column, so |uhat|^2 is the
+// quadratic Qa + jc (Qb + jc Qc) in jc, and S1, S2, S11, S12, S22 follow
+// exactly (up to rounding) from M0 = sum v, MY = sum jc v, MYY = sum jc^2 v:
+//   S_j  = U_j M0 + beta_j MY,
+//   S_jl = U_l (U_j M0 + beta_j MY) + beta_l (U_j MY + beta_j MYY).
+// That takes three accumulations per pixel instead of seven.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float2 f2fma(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 __device__ __forceinline__ float2 f2mul(float2 a, float2 b) { return __fmul2_rn(a, b); }
@@ -470,53 +477,50 @@ struct PairShape {
     static constexpr int R = (K - 1) / 2;
     static constexpr int NPW = (K + 1) / 2;                  // pairs per window row
     static constexpr int SLOTS = NPW * K;                    // pair slots per window
-    // Lane l takes pair column l % NPW of rows l / NPW, l / NPW + RPS, ...;
-    // when NPW does not divide 8, lanes NPW .. 7 idle.
-    static constexpr int RPS = (kGroup % NPW) == 0 ? kGroup / NPW : 1;  // rows per lane step
-    static constexpr int LANES = RPS * NPW;                  // active lanes of a group
-    static constexpr int NS = (K + RPS - 1) / RPS;           // rows (slots) per active lane
     static constexpr int NP4 = C / 2;                        // float4 planes (two channels each)
     static constexpr int NP2 = C & 1;                        // float2 plane (the odd channel)
     static constexpr int ROWS = kTile + 2 * R;               // staged rows: the tile and its apron
-    static constexpr int PAIRS = kTile / 2 + R;              // staged pairs per row and parity
-    static constexpr int PITCH = PAIRS + (((NPW - PAIRS) % 8) + 8) % 8;
-    static constexpr int PLANE = ROWS * PITCH;               // elements per (parity, plane)
+    // Staged columns X0 - 8 .. X0 + 23: every pair a home window reads (its
+    // first pair starts at X0 - r - 1 or later, its last ends at X0 + 16 + r
+    // or earlier).
+    static constexpr int XOFF = 8;
+    static constexpr int PAIRS = kTile / 2 + XOFF;           // staged pairs per row
+    static constexpr int PITCH = PAIRS;
+    static constexpr int PLANE = ROWS * PITCH;               // elements per plane
     static constexpr int NIT = ROWS * PAIRS;                 // staging items
     static constexpr int RV = HRec<C>::RV;
-    static constexpr size_t HALO4 = sizeof(float4) * 2 * NP4 * PLANE;
-    static constexpr size_t HALO2 = sizeof(float2) * 2 * NP2 * PLANE;
+    static constexpr size_t HALO4 = sizeof(float4) * NP4 * PLANE;
+    static constexpr size_t HALO2 = sizeof(float2) * NP2 * PLANE;
+    static_assert(R < XOFF, "window apron within the staged columns");
     // Dynamic shared memory for a record capacity of rcap home Gaussians.
     __host__ __device__ static constexpr size_t smem(int rcap) { return HALO4 + HALO2 + sizeof(float4) * RV * rcap; }
 };
 
-// Stages dL/dI of the pair kernels' region [X0 - r, X0 + 15 + r] x rows
-// [Y0 - r, Y0 + 15 + r] (zero outside it and outside the grid) for rows of a
-// multiple of 4 elements and an image aligned to 4 elements: thread (row, j)
-// loads the aligned 4 elements of columns X0 - 8 + 4j .. + 3 of every channel
-// (one vector load each: a float4, or 8 bytes of fp16 / bf16 widened to fp32;
-// guarded scalar loads where it crosses the grid's edge) and writes the
-// parity elements whose first pixel it holds, the second pixel of a pair that
-// ends past its 4 elements coming from the next lane (the group to its right).
+// Stages dL/dI of the pair kernels' region, rows [Y0 - r, Y0 + 15 + r] and
+// the pairs of columns X0 - 8 .. X0 + 23, zero outside [X0 - r, X0 + 15 + r]
+// and outside the grid, for rows of a multiple of 4 elements and an image
+// aligned to 4 elements: item (row, j) loads the aligned 4 elements from
+// X0 - 8 + 4j of every channel (one vector load each: a float4, or 8 bytes of
+// fp16 / bf16 widened to fp32; guarded scalar loads where it crosses the
+// grid's edge) and writes staged pairs 2j and 2j + 1.
 template <int C, int K, int NT, bool HALF>
 __device__ __forceinline__ void stage_pairs_vec4(const void *__restrict__ gimg, const Geom &g,
                                                  int b, int X0, int Y0, float4 *halo4,
                                                  float2 *halo2) {
     using S = PairShape<C, K, NT>;
     constexpr int R = S::R, NP4 = S::NP4, NP2 = S::NP2;
-    constexpr int NJ = (8 + kTile + R + 1 + 3) / 4;  // float4 columns from X0 - 8
-    static_assert(NJ == 8 && R <= 8, "one warp covers 4 rows of 8 float4 columns");
+    constexpr int NJ = S::PAIRS / 2;  // float4 columns per row
     constexpr int NCH = 2 * NP4 + NP2;
-    for (int it0 = 0; it0 < S::ROWS * NJ; it0 += NT) {  // every lane runs every round (shuffle)
-        const int it = it0 + (int)threadIdx.x;
+    for (int it = (int)threadIdx.x; it < S::ROWS * NJ; it += NT) {
         const int row = it / NJ, j = it - row * NJ;
         const int y = Y0 - R + row;
-        const int x4 = X0 - 8 + 4 * j;
+        const int x4 = X0 - S::XOFF + 4 * j;
         float v[NCH][4];
-        const bool rowin = row < S::ROWS && y >= 0 && y < g.H;
+        const bool rowin = y >= 0 && y < g.H;
 #pragma unroll
         for (int c = 0; c < NCH; ++c) {
             v[c][0] = v[c][1] = v[c][2] = v[c][3] = 0.0f;
-            if (c < C && rowin) {
+            if (rowin) {
                 const size_t row0 = (((size_t)b * C + c) * g.H + y) * g.W;
                 if (x4 >= 0 && x4 + 3 < g.W) {
                     if constexpr (!HALF) {
@@ -537,47 +541,24 @@ __device__ __forceinline__ void stage_pairs_vec4(const void *__restrict__ gimg, 
                         if (x4 + e >= 0 && x4 + e < g.W) v[c][e] = img_load(gimg, row0 + x4 + e, g.img_dtype);
                 }
             }
-            // zero outside [X0 - r, X0 + 15 + r]
 #pragma unroll
             for (int e = 0; e < 4; ++e)
                 if (x4 + e < X0 - R || x4 + e > X0 + kTile - 1 + R) v[c][e] = 0.0f;
         }
-        // Element 0 of the float4 to the right: the next lane's (j + 1 of the
-        // same row, NT and NJ being multiples of 8).  For j = 7 it is never
-        // used: the last pair of either parity ends inside that float4.
-        float nx[NCH];
+        const int el = row * S::PITCH + 2 * j;
 #pragma unroll
-        for (int c = 0; c < NCH; ++c) nx[c] = __shfl_down_sync(0xffffffffu, v[c][0], 1);
-        if (row >= S::ROWS) continue;
-        // Plane parity p's element m starts at column offset (8 - r) + p + 2m
-        // from X0 - 8; this float4 holds offsets 4j .. 4j + 3.
+        for (int h = 0; h < 2; ++h) {
 #pragma unroll
-        for (int p = 0; p < 2; ++p) {
-#pragma unroll
-            for (int f = 0; f < 4; ++f) {
-                if (((8 - R + p) & 1) != (f & 1)) continue;  // pairs start at this parity
-                const int m = (4 * j + f - (8 - R + p)) / 2;
-                if (4 * j + f - (8 - R + p) < 0 || m >= S::PAIRS) continue;
-                const int el = row * S::PITCH + m;
-#pragma unroll
-                for (int pl = 0; pl < NP4; ++pl) {
-                    const float lo0 = v[2 * pl][f], lo1 = v[2 * pl + 1][f];
-                    const float hi0 = f < 3 ? v[2 * pl][f < 3 ? f + 1 : 0] : nx[2 * pl];
-                    const float hi1 = f < 3 ? v[2 * pl + 1][f < 3 ? f + 1 : 0] : nx[2 * pl + 1];
-                    halo4[(p * NP4 + pl) * S::PLANE + el] = make_float4(lo0, hi0, lo1, hi1);
-                }
-                if constexpr (NP2) {
-                    const float lo = v[C - 1][f];
-                    const float hi = f < 3 ? v[C - 1][f < 3 ? f + 1 : 0] : nx[C - 1];
-                    halo2[p * S::PLANE + el] = make_float2(lo, hi);
-                }
-            }
+            for (int pl = 0; pl < NP4; ++pl)
+                halo4[pl * S::PLANE + el + h] = make_float4(v[2 * pl][2 * h], v[2 * pl][2 * h + 1],
+                                                            v[2 * pl + 1][2 * h], v[2 * pl + 1][2 * h + 1]);
+            if constexpr (NP2) halo2[el + h] = make_float2(v[C - 1][2 * h], v[C - 1][2 * h + 1]);
         }
     }
 }
 
 template <int C, int K, int NT>
-__global__ void __launch_bounds__(NT, 896 / NT) k_bwd_pairs(const float *__restrict__ params,
+__global__ void __launch_bounds__(NT, 1024 / NT) k_bwd_pairs(const float *__restrict__ params,
                                                   const void *__restrict__ gimg, Geom g,
                                                   const float4 *__restrict__ gr,
                                                   const int *__restrict__ offs,
@@ -585,15 +566,15 @@ __global__ void __launch_bounds__(NT, 896 / NT) k_bwd_pairs(const float *__restr
                                                   float *__restrict__ dparams,
                                                   int *__restrict__ err) {
     using S = PairShape<C, K, NT>;
-    constexpr int R = S::R, NPW = S::NPW, NS = S::NS, NP4 = S::NP4, NP2 = S::NP2;
+    constexpr int R = S::R, NPW = S::NPW, NP4 = S::NP4, NP2 = S::NP2;
     constexpr int RV = S::RV, NG = NT / kGroup;
     constexpr int NCH = 2 * NP4 + NP2;  // channels staged per pixel (C, rounded to the planes)
     extern __shared__ float4 smem4[];
     __shared__ int wcnt[2 * kPer * NT / 32];
     const int rcap = g.bwd_rcap;  // home records staged at most
-    float4 *halo4 = smem4;                                             // [parity][NP4][ROWS][PITCH]
-    float2 *halo2 = reinterpret_cast<float2 *>(smem4 + 2 * NP4 * S::PLANE);  // [parity][ROWS][PITCH]
-    float4 *recs = smem4 + (S::HALO4 + S::HALO2) / sizeof(float4);    // [rcap][RV]
+    float4 *halo4 = smem4;                                                // [NP4][ROWS][PITCH]
+    float2 *halo2 = reinterpret_cast<float2 *>(smem4 + NP4 * S::PLANE);  // [ROWS][PITCH]
+    float4 *recs = smem4 + (S::HALO4 + S::HALO2) / sizeof(float4);       // [rcap][RV]
     static_assert(S::HALO2 % sizeof(float4) == 0, "record area must stay 16-byte aligned");
     if (dynamic_smem_bytes() < (unsigned)S::smem(rcap) || g.k != K || rcap < NT) {
         if (threadIdx.x == 0) atomicOr(err, kErrSmemLayout);  // launch/layout mismatch
@@ -603,7 +584,7 @@ __global__ void __launch_bounds__(NT, 896 / NT) k_bwd_pairs(const float *__restr
     const int b = blockIdx.x / g.T, t = blockIdx.x - b * g.T;
     const int ty = t / g.TX, tx = t - ty * g.TX;
     const int X0 = tx * kTile, Y0 = ty * kTile;
-    const int RX0 = X0 - R, RY0 = Y0 - R;  // staged region origin (grid coordinates)
+    const int SX0 = X0 - S::XOFF, RY0 = Y0 - R;  // staged region origin (grid coordinates)
     const int tid = threadIdx.x;
     const int grp = tid / kGroup, lig = tid % kGroup;
     const unsigned gmask = ((1u << kGroup) - 1u) << (kGroup * (grp % (32 / kGroup)));
@@ -622,14 +603,13 @@ __global__ void __launch_bounds__(NT, 896 / NT) k_bwd_pairs(const float *__restr
         else
             stage_pairs_vec4<C, K, NT, true>(gimg, g, b, X0, Y0, halo4, halo2);
     } else {
-        // Stage dL/dI over [X0 - r, X0 + 15 + r]^2 (zero outside the grid; the
-        // column after it, read only as the masked pixel of a last pair, is zero
-        // too): item (row, m) holds pixels RX0 + 2m + {0, 1, 2}; the even parity
-        // gets pair (0, 1), the odd parity pair (1, 2).  Two items per thread
-        // have their loads in flight together.
+        // The same region element by element: item (row, m) holds pixels
+        // SX0 + 2m and SX0 + 2m + 1 (zero outside [X0 - r, X0 + 15 + r] and
+        // outside the grid).  Two items per thread have their loads in
+        // flight together.
         constexpr int SU = 2;
         for (int i0 = 0; i0 < S::NIT; i0 += SU * NT) {
-            float v[SU][3][NCH];
+            float v[SU][2][NCH];
 #pragma unroll
             for (int u = 0; u < SU; ++u) {
                 const int it = i0 + u * NT + tid;
@@ -637,9 +617,9 @@ __global__ void __launch_bounds__(NT, 896 / NT) k_bwd_pairs(const float *__restr
                 const int y = RY0 + row;
                 const bool rowin = it < S::NIT && y >= 0 && y < g.H;
 #pragma unroll
-                for (int q = 0; q < 3; ++q) {
-                    const int x = RX0 + 2 * m + q;
-                    const bool in = rowin && x >= 0 && x < g.W && x <= X0 + kTile - 1 + R;
+                for (int q = 0; q < 2; ++q) {
+                    const int x = SX0 + 2 * m + q;
+                    const bool in = rowin && x >= 0 && x < g.W && x >= X0 - R && x <= X0 + kTile - 1 + R;
 #pragma unroll
                     for (int c = 0; c < NCH; ++c)
                         v[u][q][c] = (in && c < C) ? img_load(gimg, (((size_t)b * C + c) * g.H + y) * g.W + x, g.img_dtype) : 0.0f;
@@ -652,35 +632,24 @@ __global__ void __launch_bounds__(NT, 896 / NT) k_bwd_pairs(const float *__restr
                 const int row = it / S::PAIRS, m = it - row * S::PAIRS;
                 const int el = row * S::PITCH + m;
 #pragma unroll
-                for (int pl = 0; pl < NP4; ++pl) {
+                for (int pl = 0; pl < NP4; ++pl)
                     halo4[pl * S::PLANE + el] = make_float4(v[u][0][2 * pl], v[u][1][2 * pl],
                                                             v[u][0][2 * pl + 1], v[u][1][2 * pl + 1]);
-                    halo4[(NP4 + pl) * S::PLANE + el] = make_float4(v[u][1][2 * pl], v[u][2][2 * pl],
-                                                                    v[u][1][2 * pl + 1], v[u][2][2 * pl + 1]);
-                }
-                if constexpr (NP2) {
-                    halo2[el] = make_float2(v[u][0][C - 1], v[u][1][C - 1]);
-                    halo2[S::PLANE + el] = make_float2(v[u][1][C - 1], v[u][2][C - 1]);
-                }
+                if constexpr (NP2) halo2[el] = make_float2(v[u][0][C - 1], v[u][1][C - 1]);
             }
         }
     }
 
     zero_missing(gr, g, b, t, dparams);
 
-    // This lane's pair column and first row (independent of the Gaussian),
-    // with the mask of the pair's second pixel (last pair of a row).
-    // With one row per lane step (RPS == 1) every active lane starts on row 0
-    // and its last row is the window's last; with all 8 lanes active (k = 15)
-    // no lane idles: both tests are then compile-time constants.
-    constexpr bool kAllOn = S::LANES == kGroup;
-    const bool lane_on = kAllOn || lig < S::LANES;
-    const int pc = lig % NPW, r0 = S::RPS == 1 ? 0 : lig / NPW;
-    const float2 sfx = make_float2((float)(2 * pc), (float)(2 * pc + 1));
-    const float2 sfy = f2dup((float)r0);
-    const float smask = pc == NPW - 1 ? __int_as_float(0x7f800000) : 0.0f;  // +inf: 2^-inf = 0
-    const int soff = r0 * S::PITCH + pc;
-    const bool last_ok = S::RPS == 1 || r0 + (NS - 1) * S::RPS < K;  // the lane's last row lies in the window
+    // This lane's pair column (independent of the Gaussian).  A lane walks
+    // every row of its column; with all 8 lanes active (k = 15) no lane idles
+    // and the test is a compile-time constant.
+    constexpr bool kAllOn = NPW == kGroup;
+    static_assert(NPW <= kGroup, "one pair column per lane");
+    const bool lane_on = kAllOn || lig < NPW;
+    const int pc = lig % NPW;
+    const float kInf = __int_as_float(0x7f800000);  // 2^-inf = 0: a masked pixel
 
     // The staged home Gaussians recs[0 .. n), one per group at a time.
     auto process = [&](int n) {
@@ -726,30 +695,62 @@ __global__ void __launch_bounds__(NT, 896 / NT) k_bwd_pairs(const float *__restr
 
             const bool ongrid = __float_as_int(q2.w) != 0;
             if (ongrid && lane_on) {
-                const float4 *hp4 = halo4 + __float_as_int(q2.x) + soff;
-                const float2 *hp2 = halo2 + __float_as_int(q2.y) + soff;
-                float2 u1 = f2fma(A1, sfx, f2fma(B1, sfy, K1));
-                float2 u2 = f2fma(A2, sfx, f2fma(B2, sfy, K2));
-                const float2 RB1 = S::RPS == 1 ? B1 : f2mul(B1, f2dup((float)S::RPS));
-                const float2 RB2 = S::RPS == 1 ? B2 : f2mul(B2, f2dup((float)S::RPS));
+                // Row moments of the lane's column (see the section comment).
+                // par = 1: the window starts at odd x and its pairs one pixel
+                // before it, so the pixel offsets of the lane's pair are
+                // 2 pc - 1 and 2 pc, and lane 0's first pixel is masked;
+                // par = 0: offsets 2 pc and 2 pc + 1, the last lane's second
+                // pixel masked.
+                const int el = __float_as_int(q2.x), par = __float_as_int(q2.y);
+                const float4 *hp4 = halo4 + el + pc;
+                const float2 *hp2 = halo2 + el + pc;
+                const float2 sfx = make_float2((float)(2 * pc - par), (float)(2 * pc + 1 - par));
+                const float2 U1 = f2fma(A1, sfx, f2fma(B1, f2dup((float)R), K1));
+                const float2 U2 = f2fma(A2, sfx, f2fma(B2, f2dup((float)R), K2));
+                float2 Qa = f2fma(U1, U1, f2mul(U2, U2));
+                if (par) {
+                    if (pc == 0) Qa.x = kInf;
+                } else if (pc == NPW - 1) {
+                    Qa.y = kInf;
+                }
+                const float2 Qb = f2mul(f2dup(2.0f), f2fma(U1, B1, f2mul(U2, B2)));
+                const float2 Qc = f2dup(fmaf(q0.y, q0.y, q1.x * q1.x));
+                float2 M0 = z2, MY = z2, MYY = z2;
 #pragma unroll
-                for (int j = 0; j < NS; ++j) {
-                    if (j > 0) {
-                        u1 = f2add(u1, RB1);
-                        u2 = f2add(u2, RB2);
+                for (int j = 0; j < K; ++j) {
+                    const int jc = j - R;
+                    const float2 JC = f2dup((float)jc);
+                    float2 gc[C];
+#pragma unroll
+                    for (int pl = 0; pl < NP4; ++pl) {
+                        const float4 P = hp4[j * S::PITCH + pl * S::PLANE];
+                        gc[2 * pl] = make_float2(P.x, P.y);
+                        gc[2 * pl + 1] = make_float2(P.z, P.w);
                     }
-                    if (j < NS - 1 || last_ok) {
-                        float2 gc[C];
+                    if constexpr (NP2) gc[C - 1] = hp2[j * S::PITCH];
+                    const float2 q = jc == 0 ? Qa : f2fma(f2fma(Qc, JC, Qb), JC, Qa);
+                    const float2 w = make_float2(ex2(-q.x), ex2(-q.y));
+                    float2 G = f2mul(gc[0], AMP[0]);
 #pragma unroll
-                        for (int pl = 0; pl < NP4; ++pl) {
-                            const float4 P = hp4[j * S::RPS * S::PITCH + pl * S::PLANE];
-                            gc[2 * pl] = make_float2(P.x, P.y);
-                            gc[2 * pl + 1] = make_float2(P.z, P.w);
-                        }
-                        if constexpr (NP2) gc[C - 1] = hp2[j * S::RPS * S::PITCH];
-                        slot(u1, u2, smask, gc);
+                    for (int c = 1; c < C; ++c) G = f2fma(gc[c], AMP[c], G);
+#pragma unroll
+                    for (int c = 0; c < C; ++c) DA[c] = f2fma(gc[c], w, DA[c]);
+                    const float2 v = f2mul(w, G);
+                    M0 = f2add(M0, v);
+                    if (jc != 0) {
+                        MY = f2fma(v, JC, MY);
+                        MYY = f2fma(v, f2dup((float)(jc * jc)), MYY);
                     }
                 }
+                const float2 t1 = f2fma(B1, MY, f2mul(U1, M0));   // sum v uhat_1
+                const float2 t2 = f2fma(B2, MY, f2mul(U2, M0));   // sum v uhat_2
+                const float2 r1 = f2fma(B1, MYY, f2mul(U1, MY));  // sum v jc uhat_1
+                const float2 r2 = f2fma(B2, MYY, f2mul(U2, MY));  // sum v jc uhat_2
+                S1 = t1;
+                S2 = t2;
+                S11 = f2fma(B1, r1, f2mul(U1, t1));
+                S12 = f2fma(B2, r1, f2mul(U2, t1));
+                S22 = f2fma(B2, r2, f2mul(U2, t2));
             } else if (!ongrid) {
                 // Centred off the grid: read dL/dI from global memory, zero
                 // outside the grid (rare: a centre within r of the border).
@@ -807,11 +808,9 @@ __global__ void __launch_bounds__(NT, 896 / NT) k_bwd_pairs(const float *__restr
         home_record_common<C>(params, gr, g, b, id, cx, cy, Rr);
         const int wx0 = cx - R, wy0 = cy - R;
         const bool ongrid = cx >= 0 && cx < g.W && cy >= 0 && cy < g.H;
-        const int lx = wx0 - RX0;  // in [0, 15] on the grid
-        const int el = (wy0 - RY0) * S::PITCH + (lx >> 1);
-        Rr[2] = ongrid ? make_float4(__int_as_float((lx & 1) * NP4 * S::PLANE + el),
-                                     __int_as_float((lx & 1) * S::PLANE + el), 0.0f,
-                                     __int_as_float(1))
+        const int par = wx0 & 1;
+        const int el = (wy0 - RY0) * S::PITCH + ((wx0 - par - SX0) >> 1);  // first staged pair
+        Rr[2] = ongrid ? make_float4(__int_as_float(el), __int_as_float(par), 0.0f, __int_as_float(1))
                        : make_float4(__int_as_float(wx0), __int_as_float(wy0), 0.0f,
                                      __int_as_float(0));
 #pragma unroll
