@@ -249,9 +249,13 @@ __device__ __forceinline__ void load_gpix(const float *gh, int pix, float (&gv)[
 }
 
 // ---------------------------------------------------------------------------
-// Scalar backward (any C, any k; common k compiled in).  Eight lanes stride
-// over a Gaussian's k*k window pixels (lane l takes pixels l, l + 8, ... in
-// row-major order, from a per-block offset table).  dL/dI is staged over
+// Scalar backward (any C, any k; common k compiled in).  Eight lanes share a
+// Gaussian's k*k window.  For k = 7, 9, 11 (compiled in, C <= 4) lane l walks
+// window column l (l < min(k, 8)) and forms the column's share of the five
+// sums from its row moments, as the pixel-pair kernel does (see there); the
+// pixels of columns 8 .. k - 1 are dealt to the lanes in row-major order from
+// a per-block offset table.  For every other k the lanes stride over all the
+// window's pixels that way (lane l takes pixels l, l + 8, ...).  dL/dI is staged over
 // [X0 - 2r, X0 + 15 + 2r]^2, zero outside the core [X0 - r, X0 + 15 + r]^2
 // and outside the grid: the core holds the whole window of every home
 // Gaussian centred on the grid, and the outer ring is only read by home
@@ -315,10 +319,17 @@ __global__ void __launch_bounds__(NT, C > 4 ? 1 : 1024 / NT) k_bwd(const float *
     zero_missing(gr, g, b, t, dparams);
 
     // Window enumeration table: lane l of a group takes window pixels
-    // l, l + 8, l + 16, ... in row-major order.
-    for (int j = tid; j < (full + 1) * kGroup; j += NT) {
-        const int p = j < kk ? j : 0;
-        const int ox = p % k, oy = p / k;
+    // l, l + 8, l + 16, ... in row-major order -- with column moments, only
+    // the pixels of columns 8 .. k - 1 (XW wide), the others being walked by
+    // column.
+    constexpr bool kCols = KT >= 7 && KT <= 11;
+    constexpr int XW = kCols ? (KT > kGroup ? KT - kGroup : 0) : 0;
+    const int tabn = kCols ? XW * k : kk;  // pixels enumerated by the table
+    const int tfull = tabn / kGroup, ttail = tabn - tfull * kGroup;
+    for (int j = tid; j < (tfull + 1) * kGroup; j += NT) {
+        const int p = j < tabn ? j : 0;
+        const int ox = kCols ? kGroup + p % (XW > 0 ? XW : 1) : p % k;
+        const int oy = kCols ? p / (XW > 0 ? XW : 1) : p / k;
         table[j] = make_float4((float)ox, (float)oy, __int_as_float(oy * RP + ox), 0.0f);
     }
     // dL/dI of the core (zero outside it and outside the grid).
@@ -397,13 +408,65 @@ __global__ void __launch_bounds__(NT, C > 4 ? 1 : 1024 / NT) k_bwd(const float *
                 load_gpix<C>(gb, __float_as_int(tb.z), gv);
                 pixel(tb.x, tb.y, gv);
             };
-            if constexpr (KT > 0) {
+            if constexpr (kCols) {
+                // Columns 8 .. k - 1 pixel by pixel, then lane l walks window
+                // column l (l < min(k, 8)) by row moments: with jc = row - r and
+                // U = uhat at the column's pixel of the centre row,
+                // uhat = U + jc (beta_1, beta_2), |uhat|^2 = Qa + jc (Qb + jc Qc),
+                // and the five sums follow from M0 = sum v, MY = sum jc v,
+                // MYY = sum jc^2 v (S_j = U_j M0 + beta_j MY,
+                // S_jl = U_l (U_j M0 + beta_j MY) + beta_l (U_j MY + beta_j MYY)).
+                if constexpr (XW > 0) {
+#pragma unroll
+                    for (int j = 0; j < tfull; ++j) eval(j);
+                    if (lig < ttail) eval(tfull);
+                }
+                constexpr int KC = KT < kGroup ? KT : kGroup;
+                constexpr int RR = (KT - 1) / 2;
+                if (KC == kGroup || lig < KC) {
+                    const float ox = (float)lig;
+                    const float U1 = fmaf(a1, ox, fmaf(b1, (float)RR, K1));
+                    const float U2 = fmaf(a2, ox, fmaf(b2, (float)RR, K2));
+                    const float Qa = fmaf(U1, U1, U2 * U2);
+                    const float Qb = 2.0f * fmaf(U1, b1, U2 * b2);
+                    const float Qc = fmaf(b1, b1, b2 * b2);
+                    float M0 = 0.0f, MY = 0.0f, MYY = 0.0f;
+                    const float *gcol = gb + lig * GP;
+#pragma unroll
+                    for (int j = 0; j < KT; ++j) {
+                        const int jc = j - RR;
+                        float gv[C];
+                        load_gpix<C>(gcol, j * RP, gv);
+                        const float q = jc == 0 ? Qa : fmaf(fmaf(Qc, (float)jc, Qb), (float)jc, Qa);
+                        const float w = ex2(-q);
+                        float G = gv[0] * amp[0];
+#pragma unroll
+                        for (int c = 1; c < C; ++c) G = fmaf(gv[c], amp[c], G);
+#pragma unroll
+                        for (int c = 0; c < C; ++c) acc[5 + c] = fmaf(gv[c], w, acc[5 + c]);
+                        const float v = w * G;
+                        M0 += v;
+                        if (jc != 0) {
+                            MY = fmaf(v, (float)jc, MY);
+                            MYY = fmaf(v, (float)(jc * jc), MYY);
+                        }
+                    }
+                    const float t1 = fmaf(b1, MY, U1 * M0), t2 = fmaf(b2, MY, U2 * M0);
+                    const float q1 = fmaf(b1, MYY, U1 * MY), q2 = fmaf(b2, MYY, U2 * MY);
+                    acc[0] += t1;
+                    acc[1] += t2;
+                    acc[2] += fmaf(b1, q1, U1 * t1);
+                    acc[3] += fmaf(b2, q1, U2 * t1);
+                    acc[4] += fmaf(b2, q2, U2 * t2);
+                }
+            } else if constexpr (KT > 0) {
 #pragma unroll 8
                 for (int j = 0; j < full; ++j) eval(j);
+                if (lig < tail) eval(full);
             } else {
                 for (int j = 0; j < full; ++j) eval(j);
+                if (lig < tail) eval(full);
             }
-            if (lig < tail) eval(full);
 
             // The chain rule is linear in the sums, so each lane applies it to
             // its own partial sums before the group reduction.

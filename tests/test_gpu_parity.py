@@ -192,12 +192,13 @@ def test_long_lists_pixel_pair_backward(W):
     check_all(p, g, H, W, k)
 
 
-@pytest.mark.parametrize("k", [13, 15])
+@pytest.mark.parametrize("k", [7, 9, 11, 13, 15])
 @pytest.mark.parametrize("s1,s2", [(-1.0, 2.0), (2.0, -1.0), (-1.5, -1.5)])
-def test_pixel_pair_backward_narrow_and_elongated(k, s1, s2):
-    """Narrow and strongly elongated Gaussians on the pixel-pair backward, which forms
-    the five sums of a window column from its row moments: the terms of that expansion
-    cancel most when the Gaussian is narrow across the column and long along it."""
+def test_backward_row_moments_narrow_and_elongated(k, s1, s2):
+    """Narrow and strongly elongated Gaussians on the backward kernels that form the five
+    sums of a window column from its row moments (the pixel-pair kernel for k = 13, 15,
+    the scalar kernel's column walk for k = 7, 9, 11): the terms of that expansion cancel
+    most when the Gaussian is narrow across the column and long along it."""
     rng = np.random.default_rng(20 + k)
     B, N, C, H, W = 2, 300, 3, 48, 64
     p = _edge_params(rng, B, N, C, H, W, k)
