@@ -155,7 +155,9 @@ __device__ __forceinline__ void warp_prefix(int T, int nw, unsigned *masks, unsi
 // ---- large frames: the slab binner ---------------------------------------
 // A slab is g.slab consecutive Gaussians of one frame (a multiple of 32):
 // counted by k_slab_count blocks of 256 threads, scattered by one warp of
-// k_slab_scatter in rounds of 32.
+// k_slab_scatter in rounds of 32.  k_slab_scan and k_slab_scatter are
+// programmatic dependent launches (each waits for its predecessor at its
+// top); none of the three releases its successor early.
 constexpr int kSlabThreads = 256;
 constexpr int kSlabWarps = 8;  // most warps (slabs) per k_slab_scatter block
 
@@ -182,6 +184,7 @@ __global__ void __launch_bounds__(kSlabThreads) k_slab_count(const float *__rest
                                                              Geom g, float4 *__restrict__ gr,
                                                              int *__restrict__ hist) {
     extern __shared__ int cnt[];  // [slabs of the block][T]
+    grid_dep_wait();
     const int T = g.T, b = blockIdx.y;
     const int span = max(g.slab, kSlabThreads), ntab = span / g.slab;
     const int s0 = blockIdx.x * ntab;  // first slab of the block
@@ -219,6 +222,7 @@ constexpr int kScanRegs = 8;
 __global__ void __launch_bounds__(1024) k_slab_scan(Geom g, int *__restrict__ hist,
                                                     int *__restrict__ tot) {
     __shared__ int part[32][33];  // [warp][tile], padded against bank conflicts
+    grid_dep_wait();
     const int b = blockIdx.y, t0 = blockIdx.x * 32;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int t = t0 + lane, T = g.T;
@@ -288,6 +292,7 @@ __global__ void __launch_bounds__(32 * kSlabWarps) k_slab_scatter(
     const int *__restrict__ tot, int *__restrict__ offs, int *__restrict__ ids,
     int *__restrict__ err) {
     extern __shared__ int ssm[];
+    grid_dep_wait();
     __shared__ int warp_tot[32];
     const int T = g.T, nwb = blockDim.x >> 5;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -382,6 +387,8 @@ __global__ void __launch_bounds__(1024) k_bin_frame(const float *__restrict__ pa
                                                     int *__restrict__ ids,
                                                     int *__restrict__ err) {
     extern __shared__ unsigned fsm[];
+    grid_dep_wait();
+    grid_dep_release();
     const int T = g.T, nw = blockDim.x >> 5;
     unsigned *masks = fsm;                                                   // [nw][T]
     int *tbase = reinterpret_cast<int *>(fsm + nw * T);                     // [T]
@@ -471,6 +478,8 @@ __global__ void __launch_bounds__(kClusterBinThreads) k_bin_cluster(
     __shared__ int tstart[MT + 1];                   // frame-relative list start per tile
     __shared__ int base[MT];                         // next slot of this chunk per tile
     __shared__ unsigned masks[NW][MT];               // per-warp lane masks of a round
+    grid_dep_wait();
+    grid_dep_release();
     cg::cluster_group cluster = cg::this_cluster();
     const int T = g.T, CS = bin_cluster_size(T);
     const int q = (int)cluster.block_rank();
@@ -574,6 +583,8 @@ __global__ void __launch_bounds__(kClusterBinThreads) k_bin_cluster(
 }
 
 __global__ void k_copy_ids(int *__restrict__ dst, const int *__restrict__ src, size_t n) {
+    grid_dep_wait();
+    grid_dep_release();
     for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
          i += (size_t)gridDim.x * blockDim.x)
         dst[i] = entry_id(src[i]);
@@ -687,16 +698,22 @@ cudaError_t launch_bin(const float *params, const Geom &g, const Workspace &ws,
     const int span = g.slab > kSlabThreads ? g.slab : kSlabThreads;
     k_slab_count<<<dim3((g.N + span - 1) / span, g.B), kSlabThreads, sc, s>>>(params, g, ws.gr,
                                                                             ws.hist);
-    k_slab_scan<<<dim3((g.T + 31) / 32, g.B), 1024, 0, s>>>(g, ws.hist, ws.tot);
+    if ((e = launch_dependent(k_slab_scan, dim3((g.T + 31) / 32, g.B), dim3(1024), 0, s, g,
+                              ws.hist, ws.tot)) != cudaSuccess)
+        return e;
     const dim3 grid((g.nslab + g.slab_warps - 1) / g.slab_warps, g.B);
     if (g.m <= 2) {
         if ((e = allow_smem(k_slab_scatter<2>, ss)) != cudaSuccess) return e;
-        k_slab_scatter<2><<<grid, 32 * g.slab_warps, ss, s>>>(g, ws.gr, ws.hist, ws.tot, ws.offs,
-                                                               ws.ids, ws.err);
+        e = launch_dependent(k_slab_scatter<2>, grid, dim3(32 * g.slab_warps), ss, s, g,
+                             (const float4 *)ws.gr, (const int *)ws.hist, (const int *)ws.tot,
+                             ws.offs, ws.ids, ws.err);
+        if (e != cudaSuccess) return e;
     } else {
         if ((e = allow_smem(k_slab_scatter<3>, ss)) != cudaSuccess) return e;
-        k_slab_scatter<3><<<grid, 32 * g.slab_warps, ss, s>>>(g, ws.gr, ws.hist, ws.tot, ws.offs,
-                                                               ws.ids, ws.err);
+        e = launch_dependent(k_slab_scatter<3>, grid, dim3(32 * g.slab_warps), ss, s, g,
+                             (const float4 *)ws.gr, (const int *)ws.hist, (const int *)ws.tot,
+                             ws.offs, ws.ids, ws.err);
+        if (e != cudaSuccess) return e;
     }
     return cudaGetLastError();
 }

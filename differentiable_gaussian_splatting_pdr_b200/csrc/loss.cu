@@ -84,6 +84,8 @@ __global__ void __launch_bounds__(kLossThreads) k_loss_coef(
     float *__restrict__ part) {
     extern __shared__ float4 lsm4[];
     CoefSmem &S = *reinterpret_cast<CoefSmem *>(lsm4);
+    grid_dep_wait();
+    grid_dep_release();
     const int tid = threadIdx.x;
     const LossTile T = loss_tile(W, H, TX, TY);
     const float *ip = img + T.base, *tp = tgt + T.base;
@@ -222,6 +224,8 @@ __global__ void __launch_bounds__(kLossThreads) k_loss_grad(
     float *__restrict__ grad) {
     extern __shared__ float4 lsm4[];
     GradSmem &S = *reinterpret_cast<GradSmem *>(lsm4);
+    grid_dep_wait();
+    grid_dep_release();
     const int tid = threadIdx.x;
     const LossTile T = loss_tile(W, H, TX, TY);
     const float *ip = img + T.base, *tp = tgt + T.base;
@@ -323,6 +327,8 @@ __global__ void __launch_bounds__(256) k_loss_final(const float *__restrict__ pa
                                                     float lam, double inv_n,
                                                     float *__restrict__ loss) {
     __shared__ double sl[256], ss[256];
+    grid_dep_wait();
+    grid_dep_release();
     const int tid = threadIdx.x;
     const int per = (nblocks + 255) / 256;
     double l = 0.0, s = 0.0;
@@ -405,13 +411,20 @@ pdr_status pdr_loss_l1_ssim(const float *image, const float *target, int B, int 
         for (int d = 0; d < kLW; ++d) taps.t[d] = (float)(v[d] / sum);
     }
     const double inv_n = 1.0 / (double)n;
-    k_loss_coef<<<(unsigned)nb, kLossThreads, sc, s>>>(image, target, H, W, TX, TY, C1, C2, taps,
-                                                       coef, n, part);
-    if (cudaGetLastError() != cudaSuccess) return PDR_ERR_CUDA;
-    k_loss_grad<<<(unsigned)nb, kLossThreads, sg, s>>>(image, target, H, W, TX, TY, lam, inv_n,
-                                                       taps, coef, n, grad_image);
-    if (cudaGetLastError() != cudaSuccess) return PDR_ERR_CUDA;
-    k_loss_final<<<1, 256, 0, s>>>(part, (int)nb, lam, inv_n, loss);
+    // Programmatic dependent launches: each kernel waits for its predecessor
+    // at its top (k_loss_final needs k_loss_coef's partial sums, complete
+    // once k_loss_grad, which waited for them, is).
+    if (launch_dependent(k_loss_coef, dim3((unsigned)nb), dim3(kLossThreads), sc, s,
+                         (const float *)image, (const float *)target, H, W, TX, TY, C1, C2, taps,
+                         coef, n, part) != cudaSuccess)
+        return PDR_ERR_CUDA;
+    if (launch_dependent(k_loss_grad, dim3((unsigned)nb), dim3(kLossThreads), sg, s,
+                         (const float *)image, (const float *)target, H, W, TX, TY, lam, inv_n,
+                         taps, (const float *)coef, n, grad_image) != cudaSuccess)
+        return PDR_ERR_CUDA;
+    if (launch_dependent(k_loss_final, dim3(1), dim3(256), 0, s, (const float *)part, (int)nb, lam,
+                         inv_n, loss) != cudaSuccess)
+        return PDR_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? PDR_OK : PDR_ERR_CUDA;
 }
 

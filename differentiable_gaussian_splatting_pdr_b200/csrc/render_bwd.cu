@@ -273,6 +273,8 @@ __global__ void __launch_bounds__(NT, C > 4 ? 1 : 1024 / NT) k_bwd(const float *
                                             const int *__restrict__ ids,
                                             float *__restrict__ dparams,
                                             int *__restrict__ err) {
+    grid_dep_wait();
+    grid_dep_release();
     constexpr int GP = GPix<C>::n;
     constexpr int NV = 5 + C;
     constexpr int RV = HRec<C>::RV;
@@ -628,6 +630,8 @@ __global__ void __launch_bounds__(NT, 1024 / NT) k_bwd_pairs(const float *__rest
                                                   const int *__restrict__ ids,
                                                   float *__restrict__ dparams,
                                                   int *__restrict__ err) {
+    grid_dep_wait();
+    grid_dep_release();
     using S = PairShape<C, K, NT>;
     constexpr int R = S::R, NPW = S::NPW, NP4 = S::NP4, NP2 = S::NP2;
     constexpr int RV = S::RV, NG = NT / kGroup;
@@ -891,8 +895,11 @@ cudaError_t launch_bwd_pairs(const float *params, const void *grad_image, const 
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    k_bwd_pairs<C, K, NT><<<g.B * g.T, NT, smem, s>>>(params, grad_image, g, ws.gr, ws.offs,
-                                                      ws.ids, grad_params, ws.err);
+    const cudaError_t e = launch_dependent(k_bwd_pairs<C, K, NT>, dim3(g.B * g.T), dim3(NT), smem,
+                                           s, params, grad_image, g, (const float4 *)ws.gr,
+                                           (const int *)ws.offs, (const int *)ws.ids,
+                                           grad_params, ws.err);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
@@ -905,8 +912,11 @@ cudaError_t launch_bwd_ck(const float *params, const void *grad_image, const Geo
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    k_bwd<C, KT, NT><<<g.B * g.T, NT, smem, s>>>(params, grad_image, g, ws.gr, ws.offs, ws.ids,
-                                                 grad_params, ws.err);
+    const cudaError_t e = launch_dependent(k_bwd<C, KT, NT>, dim3(g.B * g.T), dim3(NT), smem, s,
+                                           params, grad_image, g, (const float4 *)ws.gr,
+                                           (const int *)ws.offs, (const int *)ws.ids,
+                                           grad_params, ws.err);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -244,6 +244,8 @@ __global__ void __launch_bounds__(FwdLayout<PL>::kThreads) k_fwd(const float *__
                                                                  void *__restrict__ image,
                                                                  int *__restrict__ err) {
     __shared__ FwdSmem<C, kFwdBatch> S;
+    grid_dep_wait();
+    grid_dep_release();
     const int b = blockIdx.x / g.T, t = blockIdx.x - b * g.T;
     const int ty = t / g.TX, tx = t - ty * g.TX;
     const int X0 = tx * kTile, Y0 = ty * kTile;
@@ -275,6 +277,8 @@ __global__ void __launch_bounds__(FwdLayout<PL>::kThreads) k_fwd_cluster(
     constexpr int NT = FwdLayout<PL>::kThreads;
     constexpr int NW = NT / 32;
     __shared__ FwdSmem<C, kClusterBatch> S;
+    grid_dep_wait();
+    grid_dep_release();
     __shared__ int cnt[kClusterTiles];                 // this chunk's count per tile
     __shared__ int tab[kClusterTiles][kClusterTiles];  // tab[r][t] = count of chunk r in tile t
     __shared__ int base[kClusterTiles];                // next list slot of this chunk, per tile
@@ -497,12 +501,15 @@ cudaError_t launch_fwd_c(const float *params, const Geom &g, const Workspace &ws
     if (bin_inside)
         return g.fwd_pl == 2 ? launch_fwd_cluster<C, 2>(params, g, ws, image, s)
                              : launch_fwd_cluster<C, 4>(params, g, ws, image, s);
-    if (g.fwd_pl == 2)
-        k_fwd<C, 2><<<g.B * g.T, FwdLayout<2>::kThreads, 0, s>>>(params, g, ws.gr, ws.offs,
-                                                                 ws.ids, image, ws.err);
-    else
-        k_fwd<C, 4><<<g.B * g.T, FwdLayout<4>::kThreads, 0, s>>>(params, g, ws.gr, ws.offs,
-                                                                 ws.ids, image, ws.err);
+    const cudaError_t e =
+        g.fwd_pl == 2
+            ? launch_dependent(k_fwd<C, 2>, dim3(g.B * g.T), dim3(FwdLayout<2>::kThreads), 0, s,
+                               params, g, (const float4 *)ws.gr, (const int *)ws.offs,
+                               (const int *)ws.ids, image, ws.err)
+            : launch_dependent(k_fwd<C, 4>, dim3(g.B * g.T), dim3(FwdLayout<4>::kThreads), 0, s,
+                               params, g, (const float4 *)ws.gr, (const int *)ws.offs,
+                               (const int *)ws.ids, image, ws.err);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
