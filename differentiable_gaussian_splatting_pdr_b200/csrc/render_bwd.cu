@@ -544,10 +544,13 @@ struct PairShape {
     static constexpr int SLOTS = NPW * K;                    // pair slots per window
     static constexpr int NP4 = C / 2;                        // float4 planes (two channels each)
     static constexpr int NP2 = C & 1;                        // float2 plane (the odd channel)
-    static constexpr int ROWS = kTile + 2 * R;               // staged rows: the tile and its apron
-    // Staged columns X0 - 8 .. X0 + 23: every pair a home window reads (its
-    // first pair starts at X0 - r - 1 or later, its last ends at X0 + 16 + r
-    // or earlier).
+    // Staged rows Y0 - r - 1 .. Y0 + 16 + r and columns X0 - 8 .. X0 + 23:
+    // every pair read by the window of a home Gaussian whose centre lies in
+    // [X0 - 1, X0 + 16] x [Y0 - 1, Y0 + 16] (on the grid, or one pixel off
+    // it).  Its pairs start at x0 = cx - r or, x0 being odd, at x0 - 1 (X0 is
+    // even): at X0 - 8 or later for r <= 7, and its last pair ends at
+    // X0 + 17 + r - (r & 1) <= X0 + 23.
+    static constexpr int ROWS = kTile + 2 * R + 2;
     static constexpr int XOFF = 8;
     static constexpr int PAIRS = kTile / 2 + XOFF;           // staged pairs per row
     static constexpr int PITCH = PAIRS;
@@ -561,8 +564,8 @@ struct PairShape {
     __host__ __device__ static constexpr size_t smem(int rcap) { return HALO4 + HALO2 + sizeof(float4) * RV * rcap; }
 };
 
-// Stages dL/dI of the pair kernels' region, rows [Y0 - r, Y0 + 15 + r] and
-// the pairs of columns X0 - 8 .. X0 + 23, zero outside [X0 - r, X0 + 15 + r]
+// Stages dL/dI of the pair kernels' region, rows [Y0 - r - 1, Y0 + 16 + r]
+// and the pairs of columns X0 - 8 .. X0 + 23, zero outside [X0 - r, X0 + 15 + r]
 // and outside the grid, for rows of a multiple of 4 elements and an image
 // aligned to 4 elements: item (row, j) loads the aligned 4 elements from
 // X0 - 8 + 4j of every channel (one vector load each: a float4, or 8 bytes of
@@ -578,7 +581,7 @@ __device__ __forceinline__ void stage_pairs_vec4(const void *__restrict__ gimg, 
     constexpr int NCH = 2 * NP4 + NP2;
     for (int it = (int)threadIdx.x; it < S::ROWS * NJ; it += NT) {
         const int row = it / NJ, j = it - row * NJ;
-        const int y = Y0 - R + row;
+        const int y = Y0 - R - 1 + row;
         const int x4 = X0 - S::XOFF + 4 * j;
         float v[NCH][4];
         const bool rowin = y >= 0 && y < g.H;
@@ -651,7 +654,7 @@ __global__ void __launch_bounds__(NT, 1024 / NT) k_bwd_pairs(const float *__rest
     const int b = blockIdx.x / g.T, t = blockIdx.x - b * g.T;
     const int ty = t / g.TX, tx = t - ty * g.TX;
     const int X0 = tx * kTile, Y0 = ty * kTile;
-    const int SX0 = X0 - S::XOFF, RY0 = Y0 - R;  // staged region origin (grid coordinates)
+    const int SX0 = X0 - S::XOFF, RY0 = Y0 - R - 1;  // staged region origin (grid coordinates)
     const int tid = threadIdx.x;
     const int grp = tid / kGroup, lig = tid % kGroup;
     const unsigned gmask = ((1u << kGroup) - 1u) << (kGroup * (grp % (32 / kGroup)));
@@ -760,8 +763,8 @@ __global__ void __launch_bounds__(NT, 1024 / NT) k_bwd_pairs(const float *__rest
                 S22 = f2fma(vu2, u2, S22);
             };
 
-            const bool ongrid = __float_as_int(q2.w) != 0;
-            if (ongrid && lane_on) {
+            const bool staged = __float_as_int(q2.w) != 0;
+            if (staged && lane_on) {
                 // Row moments of the lane's column (see the section comment).
                 // par = 1: the window starts at odd x and its pairs one pixel
                 // before it, so the pixel offsets of the lane's pair are
@@ -818,9 +821,9 @@ __global__ void __launch_bounds__(NT, 1024 / NT) k_bwd_pairs(const float *__rest
                 S11 = f2fma(B1, r1, f2mul(U1, t1));
                 S12 = f2fma(B2, r1, f2mul(U2, t1));
                 S22 = f2fma(B2, r2, f2mul(U2, t2));
-            } else if (!ongrid) {
-                // Centred off the grid: read dL/dI from global memory, zero
-                // outside the grid (rare: a centre within r of the border).
+            } else if (!staged) {
+                // Centred more than one pixel off the grid: read dL/dI from
+                // global memory, zero outside the grid (rare).
                 const int wx0 = __float_as_int(q2.x), wy0 = __float_as_int(q2.y);
                 for (int sl = lig; sl < S::SLOTS; sl += kGroup) {
                     const int row = sl / NPW, pcs = sl - row * NPW;
@@ -874,10 +877,12 @@ __global__ void __launch_bounds__(NT, 1024 / NT) k_bwd_pairs(const float *__rest
         int cx, cy;
         home_record_common<C>(params, gr, g, b, id, cx, cy, Rr);
         const int wx0 = cx - R, wy0 = cy - R;
-        const bool ongrid = cx >= 0 && cx < g.W && cy >= 0 && cy < g.H;
+        // Centred on the grid or at most one pixel off it: the window lies in
+        // the staged region (its off-grid pixels are staged as zero).
+        const bool staged = cx >= -1 && cx <= g.W && cy >= -1 && cy <= g.H;
         const int par = wx0 & 1;
         const int el = (wy0 - RY0) * S::PITCH + ((wx0 - par - SX0) >> 1);  // first staged pair
-        Rr[2] = ongrid ? make_float4(__int_as_float(el), __int_as_float(par), 0.0f, __int_as_float(1))
+        Rr[2] = staged ? make_float4(__int_as_float(el), __int_as_float(par), 0.0f, __int_as_float(1))
                        : make_float4(__int_as_float(wx0), __int_as_float(wy0), 0.0f,
                                      __int_as_float(0));
 #pragma unroll
