@@ -116,6 +116,28 @@ def test_bitwise_reproducible(name):
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
 
 
+@pytest.mark.parametrize("k", [13, 15])
+@pytest.mark.parametrize("H,W", [(48, 64), (45, 50)])
+def test_pixel_pair_centres_one_pixel_off_grid(k, H, W):
+    """Window centres one pixel past every edge and corner (round(mu) = -1 or W / H), on
+    grids of whole tiles (a centre at W then lies 16 pixels into the last tile column,
+    inside the pixel-pair backward's staged rows and columns) and ragged ones, next to
+    centres two and more pixels off the grid (read from global memory)."""
+    rng = np.random.default_rng(30 + k + W)
+    B, N, C = 1, 120, 3
+    p = _edge_params(rng, B, N, C, H, W, k)
+    near = [-0.75, -0.5001, W - 0.25, W - 0.5]           # round(mu) = -1 / W
+    nearh = [-0.75, -0.5001, H - 0.25, H - 0.5]
+    inside_x, inside_y = rng.uniform(0, W, 40), rng.uniform(0, H, 40)
+    xs = np.concatenate([rng.choice(near, 40), inside_x[:20], rng.choice(near, 20)])
+    ys = np.concatenate([inside_y[:20], rng.choice(nearh, 40), rng.choice(nearh, 20)])
+    p[0, :80, 0], p[0, :80, 1] = xs[:80], ys[:80]
+    p[0, 80:100, 0] = rng.choice([-2.6, -4.0, W + 1.6, W + 3.0], 20)  # further off
+    p[0, 80:100, 1] = rng.uniform(0, H, 20)
+    g = rng.standard_normal((B, C, H, W)).astype(np.float32)
+    check_all(p, g, H, W, k)
+
+
 @pytest.mark.parametrize("name", ["tiny", "mono64", "rgb128", "field32x64", "stress512"])
 def test_graph_replay_matches_eager(name):
     """Binning, forward and backward captured in one CUDA graph (the kernels are chained
