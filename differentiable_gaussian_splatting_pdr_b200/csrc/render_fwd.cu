@@ -85,6 +85,14 @@ __device__ __forceinline__ void render_list(const Geom &g, Fetch fetch, const in
 
     const unsigned lt = lanemask_lt();
     static_assert(NB * FwdRec<C>::kVec * 16 <= 65536, "record offsets must fit 16 bits");
+    // PL = 4: |uhat|^2 over the lane's run of 4 pixels as the quadratic about
+    // the run's centre x_c = x + 1.5: with U = uhat(x_c), D = U . d uhat/dx and
+    // Qc = |d uhat / dx|^2, the pixel at x_c + o has |uhat|^2 = |U|^2 + 2 o D + o^2 Qc,
+    // o = +-0.5, +-1.5 (two operations per pixel instead of four; every term is
+    // bounded by the expansion at the run's centre).  Qc rides in the record's
+    // padding when it has a free float.
+    constexpr bool kQcRec = 6 + C < RV * 4;
+    const float fxc = fx + 0.5f * (float)(PL - 1);
     for (int e0 = 0; e0 < L; e0 += NB) {
         const int n = min(NB, L - e0);
         __syncthreads();  // the previous batch is fully consumed
@@ -112,6 +120,7 @@ __device__ __forceinline__ void render_list(const Geom &g, Fetch fetch, const in
             for (int c = 0; c < C; ++c) r[6 + c] = amp[c];
 #pragma unroll
             for (int c = 6 + C; c < RV * 4; ++c) r[c] = 0.0f;
+            if constexpr (kQcRec) r[6 + C] = fmaf(A.z, A.z, Q.x * Q.x);  // |d uhat / dx|^2
 #pragma unroll
             for (int v = 0; v < RV; ++v)
                 S.rec[e * RV + v] = make_float4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
@@ -167,18 +176,40 @@ __device__ __forceinline__ void render_list(const Geom &g, Fetch fetch, const in
                 rr[4 * v] = q.x; rr[4 * v + 1] = q.y; rr[4 * v + 2] = q.z; rr[4 * v + 3] = q.w;
             }
             const unsigned bits = pk >> bitshift;
-            float u1 = fmaf(rr[0], fx, fmaf(rr[1], fy, rr[2]));
-            float u2 = fmaf(rr[3], fx, fmaf(rr[4], fy, rr[5]));
+            if constexpr (PL == 4) {
+                const float u1 = fmaf(rr[0], fxc, fmaf(rr[1], fy, rr[2]));
+                const float u2 = fmaf(rr[3], fxc, fmaf(rr[4], fy, rr[5]));
+                const float qc = fmaf(u1, u1, u2 * u2);
+                const float D = fmaf(u1, rr[0], u2 * rr[3]);
+                float Qc;
+                if constexpr (kQcRec)
+                    Qc = rr[6 + C];
+                else
+                    Qc = fmaf(rr[0], rr[0], rr[3] * rr[3]);
+                const float s = fmaf(0.25f, Qc, qc), t = fmaf(2.25f, Qc, qc);
+                const float q[4] = {fmaf(-3.0f, D, t), s - D, s + D, fmaf(3.0f, D, t)};
 #pragma unroll
-            for (int j = 0; j < PL; ++j) {
-                if (j) {
-                    u1 += rr[0];
-                    u2 += rr[3];
+                for (int j = 0; j < 4; ++j) {
+                    const float w = ex2(-q[j]);
+                    if (bits & (1u << j)) {
+#pragma unroll
+                        for (int c = 0; c < C; ++c) acc[j][c] = fmaf(rr[6 + c], w, acc[j][c]);
+                    }
                 }
-                const float w = ex2(fmaf(-u1, u1, -u2 * u2));
-                if (bits & (1u << j)) {
+            } else {
+                float u1 = fmaf(rr[0], fx, fmaf(rr[1], fy, rr[2]));
+                float u2 = fmaf(rr[3], fx, fmaf(rr[4], fy, rr[5]));
 #pragma unroll
-                    for (int c = 0; c < C; ++c) acc[j][c] = fmaf(rr[6 + c], w, acc[j][c]);
+                for (int j = 0; j < PL; ++j) {
+                    if (j) {
+                        u1 += rr[0];
+                        u2 += rr[3];
+                    }
+                    const float w = ex2(fmaf(-u1, u1, -u2 * u2));
+                    if (bits & (1u << j)) {
+#pragma unroll
+                        for (int c = 0; c < C; ++c) acc[j][c] = fmaf(rr[6 + c], w, acc[j][c]);
+                    }
                 }
             }
         }
