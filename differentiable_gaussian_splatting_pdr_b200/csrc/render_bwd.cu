@@ -22,11 +22,13 @@
 // compacts the flagged entries in list order (ballots and a prefix over the
 // warps), and only then gathers the records of those Gaussians into shared
 // memory, each prepared once (window origin, offset into the staged halo,
-// 2 ln2 * 2 sinh(s1 - s2), amplitudes).  Eight lanes share one Gaussian;
-// their partial sums are combined with a fixed xor-shuffle tree (a segmented
-// reduction with segments of 8 lanes), and the chain rule is applied once, so
-// no per-pixel atomics and no partial-gradient buffer are needed.  Every sum
-// has a fixed order.  Block sizes (NT) are template parameters: 128-thread
+// 2 ln2 * 2 sinh(s1 - s2), amplitudes).  Eight lanes share one Gaussian; for
+// k = 7 .. 15 (C <= 4) a lane walks window columns and forms their share of
+// the five uhat sums from three row moments per column (see the pixel-pair
+// section).  The chain rule, linear in the sums, is applied by each lane to
+// its own partial sums, which are then combined with a fixed xor-shuffle tree
+// (a segmented reduction with segments of 8 lanes), so no per-pixel atomics
+// and no partial-gradient buffer are needed.  Every sum has a fixed order.  Block sizes (NT) are template parameters: 128-thread
 // blocks keep the last round of a tile's Gaussians short when a tile holds
 // few of them.
 #include "common.cuh"

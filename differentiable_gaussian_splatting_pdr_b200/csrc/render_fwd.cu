@@ -14,7 +14,8 @@
 //      window meets each of its regions, with the 16-bit mask of the region's
 //      pixels inside the window (ballot + popcount);
 //   3. evaluate: every group walks only its own sub-list; a lane evaluates
-//      its pixels from one rebased record, stepping uhat along the row.
+//      its pixels from one rebased record (PL = 4: |uhat|^2 of its run as the
+//      quadratic about the run's centre; PL = 2: stepping uhat along the row).
 // The per-pixel sum order is the list order: fixed, so results are bitwise
 // reproducible.
 //
