@@ -135,10 +135,13 @@ pdr_status check_ws(const Geom &g, void *ws, size_t bytes, Layout *L) {
 
 pdr_status from_cuda(cudaError_t e) { return e == cudaSuccess ? PDR_OK : PDR_ERR_CUDA; }
 
-// Side stream and events of pdr_step_host, one set per host thread and
-// device, created on first use and kept for the thread's lifetime.
+// Side streams and events of pdr_step_host, one set per host thread and
+// device, created on first use and kept for the thread's lifetime: `up` for
+// the dL/dI upload, `down` for the image download, so that the download can
+// run while the upload is still in flight (PCIe carries both directions at
+// once).
 struct StepSide {
-    cudaStream_t side = nullptr;
+    cudaStream_t up = nullptr, down = nullptr;
     cudaEvent_t ev[4] = {};
 };
 constexpr int kMaxDevices = 64;
@@ -150,15 +153,17 @@ cudaError_t step_side(StepSide **out) {
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
     StepSide &d = sides[dev];
-    if (!d.side) {
+    if (!d.up) {
         StepSide n;
-        e = cudaStreamCreateWithFlags(&n.side, cudaStreamNonBlocking);
+        e = cudaStreamCreateWithFlags(&n.up, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&n.down, cudaStreamNonBlocking);
         for (int j = 0; j < 4 && e == cudaSuccess; ++j)
             e = cudaEventCreateWithFlags(&n.ev[j], cudaEventDisableTiming);
         if (e != cudaSuccess) {
             for (cudaEvent_t v : n.ev)
                 if (v) cudaEventDestroy(v);
-            if (n.side) cudaStreamDestroy(n.side);
+            if (n.up) cudaStreamDestroy(n.up);
+            if (n.down) cudaStreamDestroy(n.down);
             return e;
         }
         d = n;
@@ -384,50 +389,52 @@ pdr_status pdr_step_host(const float *h_params, const float *h_grad_image, float
     StepSide *side = nullptr;
     st = from_cuda(step_side(&side));
     if (st != PDR_OK) return st;
-    cudaStream_t s2 = side->side;
+    cudaStream_t up = side->up, down = side->down;
     cudaEvent_t *ev = side->ev;
     const size_t pbytes = sizeof(float) * (size_t)B * N * g.P;
     const size_t ibytes = sizeof(float) * (size_t)B * C * H * W;
     // stream:  params H2D | forward (bins inside) | .. backward | grads D2H | join
-    // side:                 | dL/dI H2D ..         | image D2H ..
-    // The side stream starts after everything already on `stream` (ev[0]), so a
-    // previous step's backward is done with d_grad_image before it is
-    // overwritten, and `stream` joins the side stream at the end (ev[3]).
+    // up:                   | dL/dI H2D ..........|
+    // down:                                        | image D2H ......     |
+    // `up` starts after everything already on `stream` (ev[0]), so a previous
+    // step's backward is done with d_grad_image before it is overwritten; the
+    // image download starts when the forward is done (ev[2]), while the dL/dI
+    // upload may still be in flight; `stream` waits for the upload before the
+    // backward (ev[1]) and joins the download at the end (ev[3]).
     const cudaError_t e = [&]() -> cudaError_t {
         cudaError_t r;
         if (pbytes && (r = cudaMemcpyAsync(d_params, h_params, pbytes, cudaMemcpyHostToDevice, s)))
             return r;
         if ((r = cudaEventRecord(ev[0], s))) return r;
-        if ((r = cudaStreamWaitEvent(s2, ev[0], 0))) return r;
-        if ((r = cudaMemcpyAsync(d_grad_image, h_grad_image, ibytes, cudaMemcpyHostToDevice, s2)))
+        if ((r = cudaStreamWaitEvent(up, ev[0], 0))) return r;
+        if ((r = cudaMemcpyAsync(d_grad_image, h_grad_image, ibytes, cudaMemcpyHostToDevice, up)))
             return r;
-        return cudaEventRecord(ev[1], s2);
+        return cudaEventRecord(ev[1], up);
     }();
     if (e != cudaSuccess) return PDR_ERR_CUDA;
     st = pdr_render_fwd(d_params, B, N, C, H, W, k, d_image, workspace, workspace_bytes, 0,
                         stream);
-    if (st != PDR_OK) {  // still join the side stream, so that `stream` covers its copy
-        if (cudaEventRecord(ev[3], s2) == cudaSuccess) cudaStreamWaitEvent(s, ev[3], 0);
+    if (st != PDR_OK) {  // still join the upload, so that `stream` covers its copy
+        cudaStreamWaitEvent(s, ev[1], 0);
         return st;
     }
     const cudaError_t e2 = [&]() -> cudaError_t {
         cudaError_t r;
         if ((r = cudaEventRecord(ev[2], s))) return r;
-        if ((r = cudaStreamWaitEvent(s2, ev[2], 0))) return r;
-        if ((r = cudaMemcpyAsync(h_image, d_image, ibytes, cudaMemcpyDeviceToHost, s2))) return r;
-        if ((r = cudaEventRecord(ev[3], s2))) return r;
+        if ((r = cudaStreamWaitEvent(down, ev[2], 0))) return r;
+        if ((r = cudaMemcpyAsync(h_image, d_image, ibytes, cudaMemcpyDeviceToHost, down))) return r;
+        if ((r = cudaEventRecord(ev[3], down))) return r;
         return cudaStreamWaitEvent(s, ev[1], 0);
     }();
     if (e2 != cudaSuccess) return PDR_ERR_CUDA;
     st = pdr_render_bwd(d_params, d_grad_image, B, N, C, H, W, k, d_grad_params, workspace,
                         workspace_bytes, 1, stream);
-    if (st != PDR_OK) return st;
-    if (pbytes) {
+    if (st == PDR_OK && pbytes)
         st = from_cuda(cudaMemcpyAsync(h_grad_params, d_grad_params, pbytes,
                                        cudaMemcpyDeviceToHost, s));
-        if (st != PDR_OK) return st;
-    }
-    return from_cuda(cudaStreamWaitEvent(s, ev[3], 0));
+    // Join the image download whatever happened, so that `stream` covers it.
+    const pdr_status sj = from_cuda(cudaStreamWaitEvent(s, ev[3], 0));
+    return st != PDR_OK ? st : sj;
 }
 
 pdr_status pdr_check_device_error(void *workspace, void *stream) {

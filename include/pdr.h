@@ -145,10 +145,11 @@ long long pdr_list_capacity_per_frame(int N, int k);
  * h_grad_params (one cudaMemcpyAsync per buffer; pinned host memory makes
  * the copies asynchronous).  The params copy, the forward, the backward and
  * the gradient copy run on `stream`; the dL/dI copy (overlapping the forward)
- * and the image copy-back (overlapping the backward) run on a side stream of
- * the library (one per host thread and device, created on first use), which
- * starts after the work already on `stream` and which `stream` joins before
- * the call's last operation.  The call returns after enqueueing; synchronise
+ * and the image copy-back (from the end of the forward, overlapping the dL/dI
+ * copy and the backward) run on two side streams of the library (one pair per
+ * host thread and device, created on first use); the dL/dI copy starts after
+ * the work already on `stream`, and `stream` waits for it before the backward
+ * and joins the image copy-back before the call's last operation.  The call returns after enqueueing; synchronise
  * `stream` before reading h_image / h_grad_params. */
 pdr_status pdr_step_host(const float *h_params, const float *h_grad_image,
                          float *h_image, float *h_grad_params, int B, int N,
