@@ -140,9 +140,11 @@ pdr_status from_cuda(cudaError_t e) { return e == cudaSuccess ? PDR_OK : PDR_ERR
 // the dL/dI upload, `down` for the image download, so that the download can
 // run while the upload is still in flight (PCIe carries both directions at
 // once).
+constexpr int kStepChunks = 4;                       // frame chunks of a host step
+constexpr int kStepEvents = 2 + 4 * kStepChunks;
 struct StepSide {
     cudaStream_t up = nullptr, down = nullptr;
-    cudaEvent_t ev[4] = {};
+    cudaEvent_t ev[kStepEvents] = {};
 };
 constexpr int kMaxDevices = 64;
 
@@ -157,7 +159,7 @@ cudaError_t step_side(StepSide **out) {
         StepSide n;
         e = cudaStreamCreateWithFlags(&n.up, cudaStreamNonBlocking);
         if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&n.down, cudaStreamNonBlocking);
-        for (int j = 0; j < 4 && e == cudaSuccess; ++j)
+        for (int j = 0; j < kStepEvents && e == cudaSuccess; ++j)
             e = cudaEventCreateWithFlags(&n.ev[j], cudaEventDisableTiming);
         if (e != cudaSuccess) {
             for (cudaEvent_t v : n.ev)
@@ -391,50 +393,67 @@ pdr_status pdr_step_host(const float *h_params, const float *h_grad_image, float
     if (st != PDR_OK) return st;
     cudaStream_t up = side->up, down = side->down;
     cudaEvent_t *ev = side->ev;
-    const size_t pbytes = sizeof(float) * (size_t)B * N * g.P;
-    const size_t ibytes = sizeof(float) * (size_t)B * C * H * W;
-    // stream:  params H2D | forward (bins inside) | .. backward | grads D2H | join
-    // up:                   | dL/dI H2D ..........|
-    // down:                                        | image D2H ......     |
-    // `up` starts after everything already on `stream` (ev[0]), so a previous
-    // step's backward is done with d_grad_image before it is overwritten; the
-    // image download starts when the forward is done (ev[2]), while the dL/dI
-    // upload may still be in flight; `stream` waits for the upload before the
-    // backward (ev[1]) and joins the download at the end (ev[3]).
-    const cudaError_t e = [&]() -> cudaError_t {
-        cudaError_t r;
-        if (pbytes && (r = cudaMemcpyAsync(d_params, h_params, pbytes, cudaMemcpyHostToDevice, s)))
-            return r;
-        if ((r = cudaEventRecord(ev[0], s))) return r;
-        if ((r = cudaStreamWaitEvent(up, ev[0], 0))) return r;
-        if ((r = cudaMemcpyAsync(d_grad_image, h_grad_image, ibytes, cudaMemcpyHostToDevice, up)))
-            return r;
-        return cudaEventRecord(ev[1], up);
-    }();
-    if (e != cudaSuccess) return PDR_ERR_CUDA;
-    st = pdr_render_fwd(d_params, B, N, C, H, W, k, d_image, workspace, workspace_bytes, 0,
-                        stream);
-    if (st != PDR_OK) {  // still join the upload, so that `stream` covers its copy
-        cudaStreamWaitEvent(s, ev[1], 0);
-        return st;
+    // Frames are independent, so the step runs in up to kStepChunks chunks of
+    // consecutive frames, pipelined over three streams:
+    //   up:     params_c H2D, dL/dI_c H2D, for c = 0, 1, ...
+    //   stream: forward_c (bins inside) after params_c, backward_c after
+    //           dL/dI_c (reusing forward_c's bins), chunk after chunk
+    //   down:   image_c D2H after forward_c, grads_c D2H after backward_c
+    // so that the downloads of early chunks run while later chunks upload
+    // (PCIe carries both directions at once).  Every chunk's results are those
+    // of the whole batch (each frame is rendered from its own lists), and the
+    // workspace, used by one chunk at a time on `stream`, is reused.  `up`
+    // starts after everything already on `stream`, so a previous step is done
+    // with the device buffers before they are overwritten; `stream` joins both
+    // side streams before the call's last operation.
+    const int nch = B < kStepChunks ? B : kStepChunks;
+    const size_t pframe = (size_t)N * g.P, iframe = (size_t)C * H * W;  // floats per frame
+    cudaEvent_t ev_start = ev[0], ev_end = ev[1];
+    pdr_status st_out = PDR_OK;
+    cudaError_t e = cudaEventRecord(ev_start, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(up, ev_start, 0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(down, ev_start, 0);
+    for (int c = 0; c < nch && e == cudaSuccess && st_out == PDR_OK; ++c) {
+        const int b0 = (int)((long long)B * c / nch), b1 = (int)((long long)B * (c + 1) / nch);
+        const int Bc = b1 - b0;
+        cudaEvent_t ev_p = ev[2 + 4 * c], ev_g = ev[3 + 4 * c];
+        cudaEvent_t ev_f = ev[4 + 4 * c], ev_b = ev[5 + 4 * c];
+        const size_t po = (size_t)b0 * pframe, io = (size_t)b0 * iframe;
+        const size_t pbytes = sizeof(float) * (size_t)Bc * pframe;
+        const size_t ibytes = sizeof(float) * (size_t)Bc * iframe;
+        if (pbytes) e = cudaMemcpyAsync(d_params + po, h_params + po, pbytes, cudaMemcpyHostToDevice, up);
+        if (e == cudaSuccess) e = cudaEventRecord(ev_p, up);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(d_grad_image + io, h_grad_image + io, ibytes, cudaMemcpyHostToDevice, up);
+        if (e == cudaSuccess) e = cudaEventRecord(ev_g, up);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ev_p, 0);
+        if (e != cudaSuccess) break;
+        st_out = pdr_render_fwd(d_params + po, Bc, N, C, H, W, k, d_image + io, workspace,
+                                workspace_bytes, 0, stream);
+        if (st_out != PDR_OK) break;
+        e = cudaEventRecord(ev_f, s);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(down, ev_f, 0);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(h_image + io, d_image + io, ibytes, cudaMemcpyDeviceToHost, down);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ev_g, 0);
+        if (e != cudaSuccess) break;
+        st_out = pdr_render_bwd(d_params + po, d_grad_image + io, Bc, N, C, H, W, k,
+                                d_grad_params + po, workspace, workspace_bytes, 1, stream);
+        if (st_out != PDR_OK) break;
+        e = cudaEventRecord(ev_b, s);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(down, ev_b, 0);
+        if (e == cudaSuccess && pbytes)
+            e = cudaMemcpyAsync(h_grad_params + po, d_grad_params + po, pbytes,
+                                cudaMemcpyDeviceToHost, down);
     }
-    const cudaError_t e2 = [&]() -> cudaError_t {
-        cudaError_t r;
-        if ((r = cudaEventRecord(ev[2], s))) return r;
-        if ((r = cudaStreamWaitEvent(down, ev[2], 0))) return r;
-        if ((r = cudaMemcpyAsync(h_image, d_image, ibytes, cudaMemcpyDeviceToHost, down))) return r;
-        if ((r = cudaEventRecord(ev[3], down))) return r;
-        return cudaStreamWaitEvent(s, ev[1], 0);
-    }();
-    if (e2 != cudaSuccess) return PDR_ERR_CUDA;
-    st = pdr_render_bwd(d_params, d_grad_image, B, N, C, H, W, k, d_grad_params, workspace,
-                        workspace_bytes, 1, stream);
-    if (st == PDR_OK && pbytes)
-        st = from_cuda(cudaMemcpyAsync(h_grad_params, d_grad_params, pbytes,
-                                       cudaMemcpyDeviceToHost, s));
-    // Join the image download whatever happened, so that `stream` covers it.
-    const pdr_status sj = from_cuda(cudaStreamWaitEvent(s, ev[3], 0));
-    return st != PDR_OK ? st : sj;
+    // Join both side streams whatever happened, so that `stream` covers their copies.
+    cudaError_t ej = cudaEventRecord(ev_end, up);
+    if (ej == cudaSuccess) ej = cudaStreamWaitEvent(s, ev_end, 0);
+    if (ej == cudaSuccess) ej = cudaEventRecord(ev_end, down);
+    if (ej == cudaSuccess) ej = cudaStreamWaitEvent(s, ev_end, 0);
+    if (st_out != PDR_OK) return st_out;
+    if (e != cudaSuccess || ej != cudaSuccess) return PDR_ERR_CUDA;
+    return PDR_OK;
 }
 
 pdr_status pdr_check_device_error(void *workspace, void *stream) {

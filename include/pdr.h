@@ -142,14 +142,16 @@ long long pdr_list_capacity_per_frame(int N, int k);
  * copies h_params and h_grad_image to the caller's device buffers d_params and
  * d_grad_image, renders forward into d_image, runs the backward into
  * d_grad_params, and copies the image and the gradients back to h_image and
- * h_grad_params (one cudaMemcpyAsync per buffer; pinned host memory makes
- * the copies asynchronous).  The params copy, the forward, the backward and
- * the gradient copy run on `stream`; the dL/dI copy (overlapping the forward)
- * and the image copy-back (from the end of the forward, overlapping the dL/dI
- * copy and the backward) run on two side streams of the library (one pair per
- * host thread and device, created on first use); the dL/dI copy starts after
- * the work already on `stream`, and `stream` waits for it before the backward
- * and joins the image copy-back before the call's last operation.  The call returns after enqueueing; synchronise
+ * h_grad_params (cudaMemcpyAsync; pinned host memory makes the copies
+ * asynchronous).  The frames are processed in up to 4 chunks of consecutive
+ * frames, pipelined: the uploads (params, then dL/dI, chunk after chunk) run on
+ * one side stream of the library, the forward and backward of each chunk on
+ * `stream` (results bitwise those of one call over all frames; the workspace
+ * is reused chunk after chunk), and the downloads (image after the chunk's
+ * forward, gradients after its backward) on a second side stream, so that
+ * early chunks download while later ones upload.  The side streams (one pair
+ * per host thread and device, created on first use) start after the work
+ * already on `stream`, which joins both before the call's last operation.  The call returns after enqueueing; synchronise
  * `stream` before reading h_image / h_grad_params. */
 pdr_status pdr_step_host(const float *h_params, const float *h_grad_image,
                          float *h_image, float *h_grad_params, int B, int N,
