@@ -21,6 +21,10 @@ struct Layout {
     size_t err, gr, hist, tot, offs, ids, total;
 };
 
+// Forward pixels per lane: 2 for small grids (at most 2368 tiles in all:
+// more, shorter lanes per tile), else 4 (measured on B200).
+int fwd_pixels_per_lane(long long B, long long T) { return B * T <= 2368 ? 2 : 4; }
+
 pdr_status make_geom(int B, int N, int C, int H, int W, int k, Geom *g) {
     // N = 0: frames with no Gaussians (the entry points launch no kernel then).
     if (B < 1 || N < 0 || C < 1 || H < 1 || W < 1 || k < 1 || (k & 1) == 0)
@@ -79,7 +83,7 @@ pdr_status make_geom(int B, int N, int C, int H, int W, int k, Geom *g) {
     // (latency-bound); larger batches of small frames run faster as separate
     // binning and render launches (measured on B200).
     g->cluster_fwd = T <= kClusterTiles && (long long)B * T <= kClusterMaxBlocks;
-    g->fwd_pl = (long long)B * T <= 2368 ? 2 : 4;  // small grids: more, shorter lanes per tile
+    g->fwd_pl = fwd_pixels_per_lane(B, T);
     g->out_vec2 = 0;
     g->out_vec4 = 0;
     g->img_dtype = PDR_F32;
@@ -141,6 +145,7 @@ pdr_status from_cuda(cudaError_t e) { return e == cudaSuccess ? PDR_OK : PDR_ERR
 // run while the upload is still in flight (PCIe carries both directions at
 // once).
 constexpr int kStepChunks = 4;                       // frame chunks of a host step
+constexpr size_t kStepChunkMinBytes = 8u << 20;      // ... when it moves this much each way
 constexpr int kStepEvents = 2 + 4 * kStepChunks;
 struct StepSide {
     cudaStream_t up = nullptr, down = nullptr;
@@ -246,12 +251,19 @@ static bool dtype_ok(int dtype, const void *p) {
     return false;
 }
 
-pdr_status pdr_render_fwd_ex(const float *params, int B, int N, int C, int H, int W, int k,
-                             void *image, int image_dtype, void *workspace,
-                             size_t workspace_bytes, int workspace_holds_bins, void *stream) {
+namespace {
+// The forward of frames that belong to a batch of B_batch frames: the pixels
+// per lane (the one choice that changes how a pixel's weights are evaluated,
+// hence the last bits of the image) follow the whole batch, so that rendering
+// the batch in chunks gives bitwise the image of one call.
+pdr_status render_fwd_in_batch(const float *params, int B, int N, int C, int H, int W, int k,
+                               void *image, int image_dtype, void *workspace,
+                               size_t workspace_bytes, int workspace_holds_bins, void *stream,
+                               int B_batch) {
     Geom g;
     pdr_status st = make_geom(B, N, C, H, W, k, &g);
     if (st != PDR_OK) return st;
+    g.fwd_pl = fwd_pixels_per_lane(B_batch, g.T);
     if (!params_ok(g, params) || !image || !aligned4(params) || !dtype_ok(image_dtype, image))
         return PDR_ERR_INVALID_ARG;
     Layout L;
@@ -283,6 +295,14 @@ pdr_status pdr_render_fwd_ex(const float *params, int B, int N, int C, int H, in
         if (st != PDR_OK) return st;
     }
     return from_cuda(launch_fwd(params, g, ws, image, s, false));
+}
+}  // namespace
+
+pdr_status pdr_render_fwd_ex(const float *params, int B, int N, int C, int H, int W, int k,
+                             void *image, int image_dtype, void *workspace,
+                             size_t workspace_bytes, int workspace_holds_bins, void *stream) {
+    return render_fwd_in_batch(params, B, N, C, H, W, k, image, image_dtype, workspace,
+                               workspace_bytes, workspace_holds_bins, stream, B);
 }
 
 pdr_status pdr_render_fwd(const float *params, int B, int N, int C, int H, int W, int k,
@@ -406,8 +426,11 @@ pdr_status pdr_step_host(const float *h_params, const float *h_grad_image, float
     // starts after everything already on `stream`, so a previous step is done
     // with the device buffers before they are overwritten; `stream` joins both
     // side streams before the call's last operation.
-    const int nch = B < kStepChunks ? B : kStepChunks;
     const size_t pframe = (size_t)N * g.P, iframe = (size_t)C * H * W;  // floats per frame
+    // Steps that move under 8 MB each way are bound by fixed per-copy and
+    // per-launch latencies, which chunking would multiply: one chunk.
+    const bool small = sizeof(float) * (size_t)B * (pframe + iframe) < kStepChunkMinBytes;
+    const int nch = small ? 1 : (B < kStepChunks ? B : kStepChunks);
     cudaEvent_t ev_start = ev[0], ev_end = ev[1];
     pdr_status st_out = PDR_OK;
     cudaError_t e = cudaEventRecord(ev_start, s);
@@ -428,8 +451,8 @@ pdr_status pdr_step_host(const float *h_params, const float *h_grad_image, float
         if (e == cudaSuccess) e = cudaEventRecord(ev_g, up);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ev_p, 0);
         if (e != cudaSuccess) break;
-        st_out = pdr_render_fwd(d_params + po, Bc, N, C, H, W, k, d_image + io, workspace,
-                                workspace_bytes, 0, stream);
+        st_out = render_fwd_in_batch(d_params + po, Bc, N, C, H, W, k, d_image + io, PDR_F32,
+                                     workspace, workspace_bytes, 0, stream, B);
         if (st_out != PDR_OK) break;
         e = cudaEventRecord(ev_f, s);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(down, ev_f, 0);

@@ -143,8 +143,8 @@ long long pdr_list_capacity_per_frame(int N, int k);
  * d_grad_image, renders forward into d_image, runs the backward into
  * d_grad_params, and copies the image and the gradients back to h_image and
  * h_grad_params (cudaMemcpyAsync; pinned host memory makes the copies
- * asynchronous).  The frames are processed in up to 4 chunks of consecutive
- * frames, pipelined: the uploads (params, then dL/dI, chunk after chunk) run on
+ * asynchronous).  A step that moves 8 MB or more each way is processed in up
+ * to 4 chunks of consecutive frames, pipelined: the uploads (params, then dL/dI, chunk after chunk) run on
  * one side stream of the library, the forward and backward of each chunk on
  * `stream` (results bitwise those of one call over all frames; the workspace
  * is reused chunk after chunk), and the downloads (image after the chunk's

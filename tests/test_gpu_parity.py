@@ -276,12 +276,14 @@ def test_autograd_matches_direct_calls():
     assert np.array_equal(pt.grad.cpu().numpy(), dp2)
 
 
-@pytest.mark.parametrize("B", [1, 2, 5, 9])
-def test_host_step_matches_device_path(B):
-    """The host step (pipelined over chunks of frames) gives bitwise the
-    results of one device-buffer forward + backward over the whole batch,
-    also when the frames do not split evenly into chunks."""
-    w = WORKLOADS["rgb128"].scaled(B=B)
+@pytest.mark.parametrize("name,B", [("rgb128", 2), ("stress512", 1), ("stress512", 2),
+                                    ("stress512", 5)])
+def test_host_step_matches_device_path(name, B):
+    """The host step gives bitwise the results of one device-buffer forward +
+    backward over the whole batch: in one chunk (small copies), and pipelined
+    over chunks of frames (stress512-sized frames: 2 chunks, and 4 uneven ones
+    for 5 frames)."""
+    w = WORKLOADS[name].scaled(B=B)
     p, g = make_inputs(w)
     hp = torch.from_numpy(p).pin_memory()
     hg = torch.from_numpy(g).pin_memory()
