@@ -138,6 +138,36 @@ def test_pixel_pair_centres_one_pixel_off_grid(k, H, W):
     check_all(p, g, H, W, k)
 
 
+@pytest.mark.parametrize("name,B", [("mono64", 4), ("rgb128", 2), ("stress512", 1)])
+def test_render_loss_backward_chain_matches_staged(name, B):
+    """Forward, L1 + SSIM loss and backward enqueued back to back on one stream (each
+    kernel a programmatic dependent launch of the one before, the backward reading the
+    loss's dL/dI) give bitwise the results of the same calls with the stream
+    synchronised between the stages."""
+    w = WORKLOADS[name].scaled(B=B)
+    p, _ = make_inputs(w)
+    pt = torch.from_numpy(p).cuda()
+    rng = np.random.default_rng(40 + B)
+    tgt = torch.from_numpy(np.clip(rng.normal(0.5, 0.25, (B, w.C, w.H, w.W)), 0, 1)
+                           .astype(np.float32)).cuda()
+
+    def chain(staged):
+        img, ws = R.render_fwd(pt, w.H, w.W, w.k)
+        if staged:
+            torch.cuda.synchronize()
+        loss, g = R.l1_ssim_loss(img, tgt)
+        if staged:
+            torch.cuda.synchronize()
+        dp = R.render_bwd(pt, g, w.H, w.W, w.k, ws)
+        torch.cuda.synchronize()
+        R.check_device_error(ws)
+        return img, loss, g, dp
+
+    a, b = chain(False), chain(True)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
 @pytest.mark.parametrize("name", ["tiny", "mono64", "rgb128", "field32x64", "stress512"])
 def test_graph_replay_matches_eager(name):
     """Binning, forward and backward captured in one CUDA graph (the kernels are chained
